@@ -1,0 +1,317 @@
+"""Plain, slow, fp64 CPU oracle of SPADE's input-adaptive block-sparse attention.
+
+TEST INFRASTRUCTURE ONLY.  This module is what the CUDA library is checked
+against; the library itself never imports, links or calls it.  It shares no
+code with the CUDA path: the only thing both sides take from a common place is
+the seeded input generator (package spade_workloads), which holds none of the
+method's arithmetic.
+
+Source: "SPADE: An Input-Adaptive Sparse Attention Engine for Fast Video
+Diffusion Models Inference" (authors' abstract on catalyzex.com; technical
+summary on gist.science/paper/2608.03335).  The pipeline per attention head:
+
+  1. 3D tiling ("Blocking Scheme Candidates", vDiT-SSR): the latent token grid
+     (T, H, W) is cut into contiguous (bt, bh, bw) boxes.
+  2. Summarizer ("Summarizer & Estimator Expressions"): each Q/K block is
+     reduced to one d-vector; the concrete instance here is the block mean.
+  3. Estimator (same section): block-to-block importance, here the softmax
+     over key blocks of the pooled scores  Qbar_i . Kbar_j / sqrt(d).
+  4. Index search (abstract: "low-overhead index search"): per query block,
+     the smallest set of key blocks whose probability mass reaches tau, with
+     the diagonal block always kept.
+  5. Flash block-sparse attention ("Head-wise Sparse Attention Execution"):
+     exact softmax attention restricted to the kept blocks.  (Online softmax is
+     how a kernel evaluates it; the oracle evaluates the definition directly.)
+
+Readings taken where the pages are silent (each is listed in the design doc):
+  - token n = (t*H + y)*W + x; tensors [N (+text), heads, d]; batch 1;
+  - edge blocks are padded; padded keys never receive weight; padded query
+    slots produce no output; block means divide by the number of VALID tokens;
+  - the softmax over key blocks is unweighted (no block-size correction);
+  - selection: diagonal first, then the other blocks by descending probability
+    (ties -> lower block id), stopping at the first prefix whose mass >= tau;
+    tau >= 1, or a mass that never reaches tau, keeps every block;
+  - text tokens are excluded from estimation/selection; every video query also
+    attends every text key, and text queries attend every key;
+  - dense heads attend every key;
+  - softmax scale 1/sqrt(d) in both the estimator and the attention.
+
+Every function works in float64 on numpy arrays; bf16/fp32 inputs convert to
+float64 exactly.
+"""
+from __future__ import annotations
+
+import math
+from functools import lru_cache
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = [
+    "block_tokens", "valid_counts", "tile3d", "untile3d", "summarize", "estimate",
+    "select_row", "select", "selection_margin", "attention_rows", "block_sparse_attention",
+    "dense_attention", "pipeline", "kept_token_pairs",
+]
+
+
+# ---------------------------------------------------------------------------
+# 1. 3D tiling
+# ---------------------------------------------------------------------------
+
+@lru_cache(maxsize=32)
+def block_tokens(T: int, H: int, W: int, bt: int, bh: int, bw: int
+                 ) -> Tuple[Tuple[np.ndarray, np.ndarray], ...]:
+    """Per block (raster order over block-t, block-y, block-x): the token ids
+    of its valid slots and the slot numbers they occupy, both in slot order.
+
+    Slots inside a block are raster order over (t, y, x) within the box; a slot
+    whose (t, y, x) falls outside the grid is padding (vDiT-SSR, "Blocking
+    Scheme Candidates": contiguous 3D blocks of the latent grid)."""
+    nbt, nbh, nbw = -(-T // bt), -(-H // bh), -(-W // bw)
+    out = []
+    for bi in range(nbt):
+        for bj in range(nbh):
+            for bk in range(nbw):
+                toks, slots = [], []
+                for tl in range(bt):
+                    t = bi * bt + tl
+                    for yl in range(bh):
+                        y = bj * bh + yl
+                        for xl in range(bw):
+                            x = bk * bw + xl
+                            if t < T and y < H and x < W:
+                                toks.append((t * H + y) * W + x)
+                                slots.append((tl * bh + yl) * bw + xl)
+                out.append((np.asarray(toks, dtype=np.int64), np.asarray(slots, dtype=np.int64)))
+    return tuple(out)
+
+
+def valid_counts(geom: Sequence[int]) -> np.ndarray:
+    return np.asarray([len(t) for t, _ in block_tokens(*geom)], dtype=np.int64)
+
+
+def tile3d(x: np.ndarray, geom: Sequence[int]) -> np.ndarray:
+    """x [N(+text), heads, d] -> tiles [heads, nb, bt*bh*bw, d] (float64),
+    padded slots zero."""
+    T, H, W, bt, bh, bw = geom
+    blocks = block_tokens(*geom)
+    heads, d = x.shape[1], x.shape[2]
+    out = np.zeros((heads, len(blocks), bt * bh * bw, d), dtype=np.float64)
+    for b, (toks, slots) in enumerate(blocks):
+        out[:, b, slots, :] = np.transpose(x[toks].astype(np.float64), (1, 0, 2))
+    return out
+
+
+def untile3d(xt: np.ndarray, geom: Sequence[int]) -> np.ndarray:
+    """Inverse of tile3d on the valid slots: tiles -> [N, heads, d]."""
+    T, H, W = geom[:3]
+    blocks = block_tokens(*geom)
+    heads, d = xt.shape[0], xt.shape[3]
+    out = np.zeros((T * H * W, heads, d), dtype=np.float64)
+    for b, (toks, slots) in enumerate(blocks):
+        out[toks] = np.transpose(xt[:, b, slots, :], (1, 0, 2))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# 2. Summarizer: block mean over valid tokens
+# ---------------------------------------------------------------------------
+
+def summarize(x: np.ndarray, geom: Sequence[int]) -> np.ndarray:
+    """Mean of each block's valid tokens: [N, heads, d] -> [heads, nb, d]."""
+    blocks = block_tokens(*geom)
+    heads, d = x.shape[1], x.shape[2]
+    out = np.zeros((heads, len(blocks), d), dtype=np.float64)
+    for b, (toks, _) in enumerate(blocks):
+        out[:, b, :] = x[toks].astype(np.float64).sum(axis=0) / len(toks)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# 3. Estimator: softmax over key blocks of pooled scores
+# ---------------------------------------------------------------------------
+
+def estimate(qmean: np.ndarray, kmean: np.ndarray) -> np.ndarray:
+    """P[h, i, j] = softmax_j(Qbar[h,i] . Kbar[h,j] / sqrt(d))."""
+    d = qmean.shape[-1]
+    s = np.einsum("hid,hjd->hij", qmean.astype(np.float64), kmean.astype(np.float64)) / math.sqrt(d)
+    s = s - s.max(axis=-1, keepdims=True)
+    e = np.exp(s)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+# ---------------------------------------------------------------------------
+# 4. Index search: smallest diagonal-containing set reaching mass tau
+# ---------------------------------------------------------------------------
+
+def select_row(p: np.ndarray, i: int, tau: float) -> List[int]:
+    """Kept key blocks (ascending) for query block i of one head."""
+    nb = len(p)
+    if tau >= 1.0:
+        return list(range(nb))
+    kept = [i]
+    mass = float(p[i])
+    others = sorted((j for j in range(nb) if j != i), key=lambda j: (-p[j], j))
+    for j in others:
+        if mass >= tau:
+            break
+        kept.append(j)
+        mass += float(p[j])
+    return sorted(kept)
+
+
+def select(P: np.ndarray, taus: Sequence[float]) -> Tuple[np.ndarray, np.ndarray]:
+    """P [heads, nb, nb] -> (cnt [heads, nb] int32, idx [heads, nb, nb] int32,
+    row-wise ascending kept ids, unused entries -1)."""
+    heads, nb, _ = P.shape
+    cnt = np.zeros((heads, nb), dtype=np.int32)
+    idx = np.full((heads, nb, nb), -1, dtype=np.int32)
+    for h in range(heads):
+        for i in range(nb):
+            kept = select_row(P[h, i], i, float(taus[h]))
+            cnt[h, i] = len(kept)
+            idx[h, i, : len(kept)] = kept
+    return cnt, idx
+
+
+def selection_margin(p: np.ndarray, i: int, tau: float) -> float:
+    """How far row i is from changing its kept set, in probability units:
+    min(p_last_kept - p_first_dropped, tau - mass_before_last, mass_after_last - tau).
+    Rows with a small margin may legitimately differ between fp32 and fp64."""
+    nb = len(p)
+    if tau >= 1.0:
+        return math.inf
+    others = sorted((j for j in range(nb) if j != i), key=lambda j: (-p[j], j))
+    mass = float(p[i])
+    k = 0
+    prev = None
+    while mass < tau and k < len(others):
+        prev = mass
+        mass += float(p[others[k]])
+        k += 1
+    if mass < tau:            # every block kept because the mass never reached tau
+        return tau - mass
+    if k == 0:                # the diagonal alone reached tau
+        return mass - tau
+    m = min(tau - prev, mass - tau)
+    if k < len(others):
+        m = min(m, float(p[others[k - 1]] - p[others[k]]))
+    return m
+
+
+# ---------------------------------------------------------------------------
+# 5. Block-sparse attention: exact softmax attention over kept blocks
+# ---------------------------------------------------------------------------
+
+def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, head: int,
+                   rows: np.ndarray, keys: np.ndarray) -> np.ndarray:
+    """softmax(q[rows] k[keys]^T / sqrt(d)) v[keys] for one head, float64."""
+    d = q.shape[-1]
+    qq = q[rows, head, :].astype(np.float64)
+    kk = k[keys, head, :].astype(np.float64)
+    vv = v[keys, head, :].astype(np.float64)
+    s = (qq @ kk.T) / math.sqrt(d)
+    s = s - s.max(axis=1, keepdims=True)
+    e = np.exp(s)
+    return (e / e.sum(axis=1, keepdims=True)) @ vv
+
+
+def block_sparse_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+                           head_geom: Sequence[Sequence[int]],
+                           head_kept: Sequence[Optional[Sequence[Sequence[int]]]],
+                           text_tokens: int = 0,
+                           q_blocks: Optional[Dict[int, Sequence[int]]] = None) -> np.ndarray:
+    """O [N + text, heads, d] float64.
+
+    head_kept[h] is the kept-block list per query block of head h, or None for
+    a dense head.  q_blocks optionally restricts which query blocks (per head)
+    are evaluated; rows not evaluated are NaN.  Query blocks are numbered in
+    the head's scheme; for text rows use block id nb (all text rows at once)."""
+    n_tot, heads, d = q.shape
+    N = n_tot - text_tokens
+    out = np.full((n_tot, heads, d), np.nan, dtype=np.float64)
+    text = np.arange(N, n_tot, dtype=np.int64)
+    all_keys = np.arange(n_tot, dtype=np.int64)
+    for h in range(heads):
+        blocks = block_tokens(*head_geom[h])
+        nb = len(blocks)
+        want = range(nb + (1 if text_tokens else 0)) if q_blocks is None else q_blocks.get(h, [])
+        for i in want:
+            if i == nb:                                   # text query rows: dense
+                out[text, h] = attention_rows(q, k, v, h, text, all_keys)
+                continue
+            rows = blocks[i][0]
+            if head_kept[h] is None:
+                keys = all_keys
+            else:
+                parts = [blocks[j][0] for j in head_kept[h][i]]
+                if text_tokens:
+                    parts.append(text)
+                keys = np.concatenate(parts)
+            out[rows, h] = attention_rows(q, k, v, h, rows, keys)
+    return out
+
+
+def dense_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """Plain full softmax attention over every token, per head (float64)."""
+    n, heads, d = q.shape
+    out = np.empty((n, heads, d), dtype=np.float64)
+    rows = np.arange(n)
+    for h in range(heads):
+        out[:, h] = attention_rows(q, k, v, h, rows, rows)
+    return out
+
+
+def kept_token_pairs(head_geom, head_kept, text_tokens: int = 0,
+                     q_blocks: Optional[Dict[int, Sequence[int]]] = None) -> int:
+    """Number of (valid query, valid key) pairs the attention evaluates."""
+    total = 0
+    for h, geom in enumerate(head_geom):
+        vc = valid_counts(geom)
+        N = int(vc.sum())
+        nb = len(vc)
+        want = range(nb + (1 if text_tokens else 0)) if q_blocks is None else q_blocks.get(h, [])
+        for i in want:
+            if i == nb:
+                total += text_tokens * (N + text_tokens)
+            elif head_kept[h] is None:
+                total += int(vc[i]) * (N + text_tokens)
+            else:
+                total += int(vc[i]) * (int(vc[list(head_kept[h][i])].sum()) + text_tokens)
+    return total
+
+
+# ---------------------------------------------------------------------------
+# The whole path for one layer
+# ---------------------------------------------------------------------------
+
+def pipeline(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+             schemes: Sequence[Sequence[int]], head_scheme: Sequence[int],
+             head_tau: Sequence[float], head_dense: Sequence[bool],
+             text_tokens: int = 0,
+             q_blocks: Optional[Dict[int, Sequence[int]]] = None,
+             kept_override: Optional[Dict[int, Sequence[Sequence[int]]]] = None) -> dict:
+    """Steps 1-5 for every head.  Returns the per-scheme means and
+    probabilities, the kept lists and the output.  kept_override replaces the
+    oracle's own selection for the given heads (used to evaluate attention
+    under another implementation's mask)."""
+    heads = q.shape[1]
+    N = q.shape[0] - text_tokens
+    head_geom = [tuple(schemes[head_scheme[h]]) for h in range(heads)]
+    res = {"qmean": {}, "kmean": {}, "prob": {}, "kept": [None] * heads}
+    for s_id, geom in enumerate(schemes):
+        hs = [h for h in range(heads) if head_scheme[h] == s_id and not head_dense[h]]
+        if not hs:
+            continue
+        qm = summarize(q[:N, hs], geom)
+        km = summarize(k[:N, hs], geom)
+        P = estimate(qm, km)
+        res["qmean"][s_id], res["kmean"][s_id], res["prob"][s_id] = qm, km, P
+        for n, h in enumerate(hs):
+            res["kept"][h] = [select_row(P[n, i], i, float(head_tau[h])) for i in range(P.shape[1])]
+    if kept_override:
+        for h, kl in kept_override.items():
+            res["kept"][h] = [list(x) for x in kl]
+    kept = [None if head_dense[h] else res["kept"][h] for h in range(heads)]
+    res["out"] = block_sparse_attention(q, k, v, head_geom, kept, text_tokens, q_blocks)
+    return res
