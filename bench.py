@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the SPADE executor hot path on B200.
+
+One step = one whole layer through the library's grouped entry point
+(spade_grouped_attn): block means of Q and K, pooled-score estimation,
+cumulative-mass index search, cost-ranked work list and the tcgen05
+block-sparse attention, for every head of the workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan14b] [--tau 0.9]
+    python bench.py --impl reference ...      # the CPU oracle, timed on host cores
+
+Prints one JSON line (rank 0).  `value` is the effective throughput in
+TFLOP/s: 4*d FLOPs per evaluated (valid query, valid key) pair, summed over
+the whole layer and all ranks, divided by the max-over-ranks step time.
+Multi-GPU runs (torchrun) give each rank its own layer (independent layers,
+e.g. batch elements): weak scaling, no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attn effective TFLOP/s (kept-pair FLOPs / layer time), Wan-14B shape"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def _dist_env():
+    return int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Max of a float over ranks (identity when world == 1)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def assemble_line(*, value, unit, n_gpus, steps, warmup, ms, config, extra) -> dict:
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": n_gpus, "steps": steps,
+            "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config}
+    line.update(extra)
+    return line
+
+
+# ------------------------------------------------------------------ FLOPs --
+
+def kept_pair_flops(wl, kept_lists) -> int:
+    """4*d per (valid query, valid key) pair of the layer, text rows/cols included."""
+    total = 0
+    ntext = wl.text_tokens
+    for h in range(wl.heads):
+        sc = wl.schemes[wl.head_scheme[h]]
+        vc = _valid_counts(sc)
+        N = int(vc.sum())
+        kl = kept_lists[h]
+        if kl is None:
+            total += (N + ntext) * (N + ntext)
+            continue
+        csum = np.array([vc[np.asarray(k)].sum() for k in kl])
+        total += int((vc * (csum + ntext)).sum()) + ntext * (N + ntext)
+    return 4 * wl.d * total
+
+
+def _valid_counts(sc):
+    """Valid tokens per block from clipped extents (geometry only)."""
+    t = np.minimum(sc.bt, sc.T - np.arange(sc.nbt) * sc.bt)
+    y = np.minimum(sc.bh, sc.H - np.arange(sc.nbh) * sc.bh)
+    x = np.minimum(sc.bw, sc.W - np.arange(sc.nbw) * sc.bw)
+    return (t[:, None, None] * y[None, :, None] * x[None, None, :]).reshape(-1)
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        else:
+            self.out = ""
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_sample(wl, q, k, v, heads, qblocks_per_head, seed=0):
+    """Time the oracle (as it stands) on a bounded sample of the layer:
+    the full selection of `heads` heads and the attention of a few query
+    blocks of each.  Returns (seconds, flops_in_sample, sel_seconds_per_head,
+    attn_seconds, attn_flops)."""
+    import oracle as O
+    rng = np.random.default_rng(seed)
+    t_sel, t_attn, fl = 0.0, 0.0, 0
+    for h in heads:
+        sc = wl.schemes[wl.head_scheme[h]]
+        geom = sc.as_tuple()
+        qh = q[:, h: h + 1].double().cpu().numpy()
+        kh = k[:, h: h + 1].double().cpu().numpy()
+        vh = v[:, h: h + 1].double().cpu().numpy()
+        t0 = time.perf_counter()
+        if wl.head_dense[h]:
+            kept = None
+        else:
+            P = O.estimate(O.summarize(qh[: wl.N], geom), O.summarize(kh[: wl.N], geom))[0]
+            kept = [O.select_row(P[i], i, wl.head_tau[h]) for i in range(sc.nb)]
+        t1 = time.perf_counter()
+        qb = sorted(rng.choice(sc.nb, size=min(qblocks_per_head, sc.nb), replace=False).tolist())
+        t2 = time.perf_counter()
+        O.block_sparse_attention(qh, kh, vh, [geom], [kept], wl.text_tokens, {0: qb})
+        t3 = time.perf_counter()
+        fl += O.kept_token_pairs([geom], [kept], wl.text_tokens, {0: qb}) * 4 * wl.d
+        t_sel += t1 - t0
+        t_attn += t3 - t2
+    return t_sel, t_attn, fl
+
+
+def cpu_baseline(wl, q, k, v, total_flops, budget_heads=2, qblocks=3):
+    """Extrapolated oracle throughput for the whole layer (TFLOP/s)."""
+    heads = list(np.linspace(0, wl.heads - 1, budget_heads).astype(int))
+    t_sel, t_attn, fl = oracle_sample(wl, q, k, v, heads, qblocks)
+    sel_per_head = t_sel / len(heads)
+    attn_rate = fl / t_attn                           # oracle FLOP/s on attention
+    t_layer = sel_per_head * wl.heads + total_flops / attn_rate
+    cores = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:   # noqa: BLE001
+        blas = cores
+    return {"value": total_flops / t_layer / 1e12, "unit": "TFLOP/s", "cores": int(min(cores, blas)),
+            "kind": "oracle",
+            "sample": (f"selection of {len(heads)} heads + attention of {qblocks} query blocks each "
+                       f"({t_sel + t_attn:.1f} s of CPU work), extrapolated to the full layer "
+                       f"({t_layer * 1e3:.0f} ms/layer)"),
+            "ms_per_layer_extrapolated": t_layer * 1e3}
+
+
+# ------------------------------------------------------------------ main --
+
+def workload_config(wl, tau):
+    sc = wl.schemes[0]
+    return {"workload": f"{wl.name}: grid {wl.T}x{wl.H}x{wl.W} ({wl.N} tokens"
+                        f"{' + %d text' % wl.text_tokens if wl.text_tokens else ''}), {wl.heads} heads, "
+                        f"d={wl.d}, blocks " + "/".join(f"{s.bt}x{s.bh}x{s.bw}" for s in wl.schemes)
+                        + (f", tau={tau}" if tau is not None else ", per-head tau"),
+            "batch": 1, "heads": wl.heads, "d": wl.d, "tau": tau,
+            "l2": "inputs larger than L2 (Q/K/V %.2f GB)" % (3 * wl.n_total * wl.heads * wl.d * 2 / 1e9)}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, timed as it stands on host cores."""
+    import torch
+    from spade_workloads import get_config, make_qkv
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return 0
+    wl = get_config(args.config)
+    if args.tau is not None and wl.name != "mixed":
+        wl = wl.with_tau(args.tau)
+    q, k, v = make_qkv(wl, device="cpu")
+    import oracle as O
+    # estimate the whole layer's kept-pair FLOPs from the oracle's own selection on sampled heads
+    per_step = []
+    for step in range(args.warmup + args.steps):
+        heads = [int((step * 7) % wl.heads)]
+        t_sel, t_attn, fl = oracle_sample(wl, q, k, v, heads, 1, seed=step)
+        if step >= args.warmup:
+            per_step.append((t_sel, t_attn, fl))
+    t_sel = sum(x[0] for x in per_step)
+    t_attn = sum(x[1] for x in per_step)
+    fl = sum(x[2] for x in per_step)
+    value = fl / (t_sel + t_attn) / 1e12
+    cores = len(os.sched_getaffinity(0))
+    ms = (t_sel + t_attn) / len(per_step) * 1e3
+    line = assemble_line(value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+                         ms=ms, config=workload_config(wl, args.tau if wl.name != "mixed" else None),
+                         extra={"impl": "reference",
+                                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
+                                                 "kind": "oracle",
+                                                 "sample": "per step: full selection of one head + "
+                                                           "attention of one of its query blocks"},
+                                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}})
+    line["dtype"] = "f64"
+    print(json.dumps(line))
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="wan14b")
+    ap.add_argument("--tau", type=float, default=0.9)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from input_adaptive_block_b200 import api
+    from spade_workloads import get_config, make_qkv
+
+    world, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    wl = get_config(args.config)
+    tau = args.tau if wl.name != "mixed" else None
+    if tau is not None:
+        wl = wl.with_tau(tau)
+    q, k, v = make_qkv(wl, device=dev)
+    schemes = [s.as_tuple() for s in wl.schemes]
+    table = [(wl.head_scheme[h], wl.head_tau[h], wl.head_dense[h]) for h in range(wl.heads)]
+    need = api.grouped_workspace_bytes(schemes, table, wl.d, wl.text_tokens)
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        api.grouped_attn(q, k, v, schemes, table, wl.text_tokens, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if api.last_device_status() != 0:
+        raise RuntimeError("device status reports a timed-out wait")
+
+    # kept lists of this layer (for the FLOP count and the attention-only timing)
+    kept = []
+    for h in range(wl.heads):
+        if wl.head_dense[h]:
+            kept.append(None)
+            continue
+        co, io = api.grouped_head_lists(schemes, table, wl.d, wl.text_tokens, h)
+        nb = wl.schemes[wl.head_scheme[h]].nb
+        cnt = ws[co: co + 4 * nb].view(torch.int32).cpu().numpy()
+        idx = ws[io: io + 4 * nb * nb].view(torch.int32).view(nb, nb).cpu().numpy()
+        kept.append([idx[i, : cnt[i]] for i in range(nb)])
+    flops = kept_pair_flops(wl, kept)
+    sparse = [h for h in range(wl.heads) if not wl.head_dense[h]]
+    kept_frac = (np.mean([np.mean([len(x) for x in kept[h]]) / wl.schemes[wl.head_scheme[h]].nb
+                          for h in sparse]) if sparse else 1.0)
+
+    # ---- timed region: K whole-layer steps ----
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = reduce_max(ms, world, dev)
+    value = world * flops / (ms * 1e-3) / 1e12
+    clocks = clk.summary()
+
+    # ---- the dominant kernel alone: attention launches over the same masks ----
+    extra = {}
+    if len(wl.schemes) == 1 and not any(wl.head_dense):
+        co, io = api.grouped_head_lists(schemes, table, wl.d, wl.text_tokens, 0)
+        nb = wl.schemes[0].nb
+        cnt_t = ws[co: co + 4 * nb * wl.heads].view(torch.int32).view(wl.heads, nb)
+        idx_t = ws[io: io + 4 * nb * nb * wl.heads].view(torch.int32).view(wl.heads, nb, nb)
+        aws = torch.empty(max(api.attn_workspace_bytes(schemes[0], wl.heads, wl.d, wl.text_tokens), 256),
+                          dtype=torch.uint8, device=dev)
+        out2 = torch.empty_like(q)
+
+        def attn():
+            api.block_sparse_attn(q, k, v, cnt_t, idx_t, schemes[0], wl.text_tokens, out=out2, workspace=aws)
+        attn()
+        torch.cuda.synchronize()
+        assert torch.equal(out, out2), "attention-only launch differs from the grouped step"
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            attn()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        attn_ms = a0.elapsed_time(a1) / args.steps
+    else:
+        attn_ms = None
+
+    peaks = _peaks()
+    if attn_ms is not None:
+        ach = flops / (attn_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "kernel": "attn_tc_kernel<128> (+ work-list build) via spade_block_sparse_attn",
+                "peak_source": f"{peaks['source']} bf16 burst (sustained {peaks['bf16_tflops_sustained']})",
+                "attn_ms": attn_ms}
+    else:
+        ach = flops / (ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "kernel": "whole grouped step (mixed schemes)", "peak_source": f"{peaks['source']} bf16 burst"}
+    extra["roofline"] = roof
+    extra["ms_per_layer"] = ms
+    extra["block_kept_fraction"] = float(kept_frac)
+    extra["block_sparsity"] = float(1.0 - kept_frac)
+    extra["layer_gflop_kept_pairs"] = flops / 1e9
+    n_runs = 0
+    for s_id in range(len(wl.schemes)):
+        hs = [h for h in range(wl.heads) if wl.head_scheme[h] == s_id and not wl.head_dense[h]]
+        if hs:
+            runs = 1 + sum(1 for a, b in zip(hs, hs[1:]) if b != a + 1)
+            n_runs += 2 * runs + 2
+    extra["gpu_launches"] = args.steps * (n_runs + 2)
+    extra["clocks"] = clocks
+
+    # ---- end to end: pinned host inputs in, host output back, every step ----
+    if not args.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+        def e2e_step():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            step()
+            oh.copy_(out, non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, min(args.steps, 5))
+        b0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b1.record(stream)
+        torch.cuda.synchronize()
+        ems = reduce_max(b0.elapsed_time(b1) / n_e2e, world, dev)
+        extra["e2e"] = {"value": world * flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+                        "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+                        "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": ems}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        extra["cpu_baseline"] = cpu_baseline(wl, q, k, v, flops)
+
+    if rank == 0:
+        line = assemble_line(value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+                             ms=ms, config=workload_config(wl, tau), extra=extra)
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,177 @@
+/*
+ * spade.h -- C ABI of the SPADE executor hot path on NVIDIA B200 (sm_100a).
+ *
+ * What it computes (SPADE: "An Input-Adaptive Sparse Attention Engine for Fast
+ * Video Diffusion Models Inference"; authors' abstract on catalyzex.com, and
+ * the technical summary on gist.science/paper/2608.03335):
+ * the input-adaptive block-sparse self-attention of one video-DiT layer.  Per
+ * attention head:
+ *   1. 3D tiling of the latent token grid (T,H,W) into (bt,bh,bw) blocks
+ *      (technical summary, Methodology 1 "Blocking Scheme Candidates");
+ *   2. a Summarizer reducing each Q/K block to one vector -- block mean
+ *      (Methodology 1, "Summarizer & Estimator Expressions");
+ *   3. an Estimator of block-to-block importance -- softmax over key blocks of
+ *      the pooled scores Qbar_i . Kbar_j / sqrt(d) (same passage);
+ *   4. the "low-overhead index search" of the executor (abstract): per query
+ *      block, the smallest set of key blocks whose probability mass reaches
+ *      tau, diagonal block always kept;
+ *   5. flash block-sparse attention over only the kept blocks, online softmax,
+ *      no dense score matrix (Methodology 3, "Flash Block-Sparse Attention");
+ * with heads of different blocking schemes run in one grouped launch
+ * (Methodology 3, "Head Grouping"; abstract, "kernel grouping").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or synchronises (except spade_last_device_status).
+ *    Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default) and
+ *    returns before it runs.
+ *  - Token order: n = (t*H + y)*W + x.  Q/K/V/O are contiguous
+ *    [n_tokens, heads, d] (batch 1).  When text_tokens > 0 the text tokens
+ *    follow the N = T*H*W video tokens: n_tokens = N + text_tokens.
+ *  - Blocks of a scheme are numbered raster-order over (block-t, block-y,
+ *    block-x); the slots of a block raster-order over (t, y, x) inside the box.
+ *    nb = ceil(T/bt)*ceil(H/bh)*ceil(W/bw); BS = bt*bh*bw.  Edge blocks are
+ *    padded: padded slots hold zeros, padded keys get no weight, padded query
+ *    slots produce no output, and block means divide by the VALID count.
+ *  - Host-side argument errors are returned synchronously and nothing is
+ *    enqueued.  Errors detected on the device (a bounded wait that ran out)
+ *    are latched in a device status word, readable with
+ *    spade_last_device_status().
+ *  - Pointers must be 16-byte aligned.  bf16 = IEEE bfloat16 bit pattern.
+ */
+#ifndef SPADE_H_
+#define SPADE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* spade_stream_t;   /* same handle as cudaStream_t */
+
+typedef enum {
+  SPADE_OK = 0,
+  SPADE_ERR_INVALID = 1,       /* bad pointer, size or shape                    */
+  SPADE_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d not 64/128)  */
+  SPADE_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed             */
+  SPADE_ERR_TIMEOUT = 4,       /* a bounded device-side wait ran out            */
+  SPADE_ERR_WORKSPACE = 5      /* workspace missing or smaller than required    */
+} spade_status;
+
+typedef enum { SPADE_F32 = 0, SPADE_BF16 = 1 } spade_dtype;
+
+/* One blocking scheme: the (T,H,W) latent grid cut into (bt,bh,bw) boxes.
+ * A dense head may use the flat scheme {1,1,N, 1,1,128}. */
+typedef struct { int32_t T, H, W, bt, bh, bw; } spade_geom;
+
+/* Row of the per-head scheme table: which scheme the head uses, its
+ * cumulative-mass threshold tau (tau >= 1 keeps every block) and whether the
+ * head is dense (attends every key; no estimation or selection). */
+typedef struct { int32_t scheme; float tau; int32_t dense; } spade_head_scheme;
+
+/* ---- step 1: 3D tiling --------------------------------------------------
+ * Methodology 1, "Blocking Scheme Candidates" (contiguous 3D blocks of the
+ * latent grid) and Methodology 3, "Kernel Fusion" (layout transformation).
+ * x  : [>= N, heads, d] token order, dtype `dt` (rows past N are ignored).
+ * xt : [heads, nb, BS, d] same dtype; padded slots written as zero.
+ * Pure data movement: bit-exact. */
+spade_status spade_tile3d(const void* x, void* xt, spade_geom g, int heads, int d,
+                          spade_dtype dt, spade_stream_t stream);
+
+/* ---- step 2: Summarizer (block mean) -------------------------------------
+ * Methodology 1, "Summarizer & Estimator Expressions" (mean reduce of a Q/K
+ * block), fused with the tiling as in Methodology 3 "Kernel Fusion": reads x
+ * in token order and never materialises tiles.
+ * x     : [>= N, heads, d] token order, dtype `dt`.
+ * xmean : [heads, nb, d] float32, mean over each block's valid tokens
+ *         (accumulated in float32). */
+spade_status spade_summarize(const void* x, float* xmean, spade_geom g, int heads, int d,
+                             spade_dtype dt, spade_stream_t stream);
+
+/* ---- step 3: Estimator ---------------------------------------------------
+ * Methodology 1, "Summarizer & Estimator Expressions" (inter-block importance).
+ * prob[h,i,j] = softmax_j( qmean[h,i,:] . kmean[h,j,:] / sqrt(d) ), float32.
+ * qmean, kmean : [heads, nb, d] float32;  prob : [heads, nb, nb] float32.
+ * Limits: 1 <= nb <= 2048, d in {64, 128}. */
+spade_status spade_estimate(const float* qmean, const float* kmean, float* prob,
+                            int heads, int nb, int d, spade_stream_t stream);
+
+/* ---- step 4: index search -----------------------------------------------
+ * Abstract, executor "low-overhead index search"; Methodology 3, ranked
+ * block-sparse representation.  Per (head h, query block i): kept set = {i},
+ * then other blocks in descending prob (ties -> lower id) until the mass
+ * (prob[h,i,i] + sum of added) >= tau[h]; tau >= 1 or a mass that never
+ * reaches tau keeps every block.  Computed in float32.
+ * prob    : [heads, nb, nb] float32 (device).
+ * tau_host: [heads] float32 HOST array, read during the call.
+ * cnt     : [heads, nb] int32 out, number of kept blocks (>= 1).
+ * idx     : [heads, nb, nb] int32 out; row (h,i) holds its cnt[h,i] kept ids in
+ *           ascending order; entries past cnt[h,i] are left untouched.
+ * Limits: nb <= 1024, heads <= 1024. */
+spade_status spade_select(const float* prob, const float* tau_host, int* cnt, int* idx,
+                          int heads, int nb, spade_stream_t stream);
+
+/* ---- step 5: flash block-sparse attention (one scheme) -------------------
+ * Methodology 3, "Flash Block-Sparse Attention": exact softmax attention of
+ * every valid query token of block i over the valid tokens of its kept key
+ * blocks (plus every text token), scale 1/sqrt(d), online softmax.  Text
+ * query rows attend every key.  Output written in token order.
+ * q,k,v   : [N + text_tokens, heads, d], dtype `dt`.
+ * out     : [N + text_tokens, heads, d], dtype `dt`; every row written.
+ * cnt,idx : from spade_select for this scheme ([heads, nb], [heads, nb, nb]);
+ *           cnt == NULL means every head is dense.
+ * workspace: device scratch of spade_attn_workspace_bytes() bytes (work list).
+ * Paths: bf16 with BS == 128 and d in {64,128} runs the tcgen05/TMEM/TMA
+ * kernel; everything else (fp32, other block sizes) the CUDA-core kernel. */
+size_t spade_attn_workspace_bytes(spade_geom g, int heads, int d, int text_tokens);
+spade_status spade_block_sparse_attn(const void* q, const void* k, const void* v, void* out,
+                                     const int* cnt, const int* idx, spade_geom g,
+                                     int heads, int d, int text_tokens, spade_dtype dt,
+                                     void* workspace, size_t ws_bytes, spade_stream_t stream);
+
+/* ---- steps 1-5 for heads of mixed schemes, one grouped attention launch ---
+ * Methodology 3, "Head Grouping"; abstract, "kernel grouping".  Runs the
+ * summarizer, estimator and index search per scheme for the non-dense heads,
+ * builds one cost-ranked work list over all heads, and runs ONE attention
+ * launch over every head.
+ * schemes : n_schemes (1..4) geometries, all with the same T*H*W = N.
+ * table   : [heads] per-head rows (host array, read during the call).
+ * workspace: device scratch of spade_grouped_workspace_bytes() bytes.
+ * Limits: heads <= 128, as for the single steps. */
+size_t spade_grouped_workspace_bytes(const spade_geom* schemes, int n_schemes,
+                                     const spade_head_scheme* table, int heads, int d,
+                                     int text_tokens);
+spade_status spade_grouped_attn(const void* q, const void* k, const void* v, void* out,
+                                const spade_geom* schemes, int n_schemes,
+                                const spade_head_scheme* table, int heads, int d,
+                                int text_tokens, spade_dtype dt,
+                                void* workspace, size_t ws_bytes, spade_stream_t stream);
+
+/* Where, inside a grouped workspace, head `head`'s kept lists live (byte
+ * offsets of its int32 cnt [nb] and idx [nb, nb] arrays); -1 for dense heads.
+ * Lets a caller read back the mask the grouped call used. */
+spade_status spade_grouped_head_lists(const spade_geom* schemes, int n_schemes,
+                                      const spade_head_scheme* table, int heads, int d,
+                                      int text_tokens, int head,
+                                      int64_t* cnt_offset, int64_t* idx_offset);
+
+/* ---- status ---------------------------------------------------------------
+ * spade_last_device_status synchronises `stream`, returns the latched device
+ * status (SPADE_OK or SPADE_ERR_TIMEOUT) and clears it. */
+spade_status spade_last_device_status(spade_stream_t stream);
+const char* spade_status_string(spade_status s);
+const char* spade_last_error_message(void);   /* detail of the last host error */
+int spade_version(void);
+
+/* Runs a kernel whose single wait can never be satisfied, bounded by
+ * timeout_ns; the device status must then read SPADE_ERR_TIMEOUT.  Exercises
+ * the bounded-wait error path without faulting or hanging the GPU. */
+spade_status spade_selftest_bounded_wait(int64_t timeout_ns, spade_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPADE_H_ */

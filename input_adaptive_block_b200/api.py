@@ -1,0 +1,168 @@
+"""PyTorch-facing binding of the C ABI (argument marshalling only).
+
+Every function here hands device pointers of caller tensors and the current
+CUDA stream to the matching `spade_*` entry point of libspade.so; all
+arithmetic happens in its CUDA kernels.  PyTorch provides memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import SpadeGeom, SpadeHeadScheme, check
+
+__all__ = [
+    "geom", "dtype_code", "tile3d", "summarize", "estimate", "select", "attn_workspace_bytes",
+    "block_sparse_attn", "grouped_workspace_bytes", "grouped_attn", "grouped_head_lists",
+    "last_device_status", "selftest_bounded_wait", "num_blocks",
+]
+
+
+def geom(g) -> SpadeGeom:
+    """(T, H, W, bt, bh, bw) tuple, Scheme, or SpadeGeom -> SpadeGeom."""
+    if isinstance(g, SpadeGeom):
+        return g
+    t = g.as_tuple() if hasattr(g, "as_tuple") else tuple(g)
+    return SpadeGeom(*[int(v) for v in t])
+
+
+def num_blocks(g) -> int:
+    gg = geom(g)
+    return -(-gg.T // gg.bt) * -(-gg.H // gg.bh) * -(-gg.W // gg.bw)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return _lib.SPADE_F32
+    if dt == torch.bfloat16:
+        return _lib.SPADE_BF16
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return t.data_ptr()
+
+
+def tile3d(x: torch.Tensor, g, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    gg = geom(g)
+    heads, d = x.shape[1], x.shape[2]
+    nb, bs = num_blocks(gg), gg.bt * gg.bh * gg.bw
+    if out is None:
+        out = torch.empty(heads, nb, bs, d, dtype=x.dtype, device=x.device)
+    check(_lib.load().spade_tile3d(_dev(x, "x"), _dev(out, "xt"), gg, heads, d, dtype_code(x.dtype),
+                                   _stream(stream)), "spade_tile3d")
+    return out
+
+
+def summarize(x: torch.Tensor, g, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    gg = geom(g)
+    heads, d = x.shape[1], x.shape[2]
+    if out is None:
+        out = torch.empty(heads, num_blocks(gg), d, dtype=torch.float32, device=x.device)
+    check(_lib.load().spade_summarize(_dev(x, "x"), _dev(out, "xmean"), gg, heads, d, dtype_code(x.dtype),
+                                      _stream(stream)), "spade_summarize")
+    return out
+
+
+def estimate(qmean: torch.Tensor, kmean: torch.Tensor, out: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    heads, nb, d = qmean.shape
+    if out is None:
+        out = torch.empty(heads, nb, nb, dtype=torch.float32, device=qmean.device)
+    check(_lib.load().spade_estimate(_dev(qmean, "qmean"), _dev(kmean, "kmean"), _dev(out, "prob"),
+                                     heads, nb, d, _stream(stream)), "spade_estimate")
+    return out
+
+
+def select(prob: torch.Tensor, taus: Sequence[float], cnt: Optional[torch.Tensor] = None,
+           idx: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    heads, nb, _ = prob.shape
+    if cnt is None:
+        cnt = torch.empty(heads, nb, dtype=torch.int32, device=prob.device)
+    if idx is None:
+        idx = torch.full((heads, nb, nb), -1, dtype=torch.int32, device=prob.device)
+    tau_arr = (ctypes.c_float * heads)(*[float(t) for t in taus])
+    check(_lib.load().spade_select(_dev(prob, "prob"), tau_arr, _dev(cnt, "cnt"), _dev(idx, "idx"),
+                                   heads, nb, _stream(stream)), "spade_select")
+    return cnt, idx
+
+
+def attn_workspace_bytes(g, heads: int, d: int, text_tokens: int = 0) -> int:
+    return int(_lib.load().spade_attn_workspace_bytes(geom(g), heads, d, text_tokens))
+
+
+def block_sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cnt: Optional[torch.Tensor],
+                      idx: Optional[torch.Tensor], g, text_tokens: int = 0, out: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    gg = geom(g)
+    heads, d = q.shape[1], q.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    need = attn_workspace_bytes(gg, heads, d, text_tokens)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    cp = _dev(cnt, "cnt") if cnt is not None else None
+    ip = _dev(idx, "idx") if idx is not None else None
+    check(_lib.load().spade_block_sparse_attn(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), cp, ip, gg, heads, d, text_tokens,
+        dtype_code(q.dtype), _dev(workspace, "workspace"), workspace.numel(), _stream(stream)),
+        "spade_block_sparse_attn")
+    return out
+
+
+def _tables(schemes, table):
+    gs = (SpadeGeom * len(schemes))(*[geom(s) for s in schemes])
+    rows = (SpadeHeadScheme * len(table))(*[SpadeHeadScheme(int(sc), float(tau), int(bool(dn)))
+                                            for sc, tau, dn in table])
+    return gs, rows
+
+
+def grouped_workspace_bytes(schemes, table, d: int, text_tokens: int = 0) -> int:
+    gs, rows = _tables(schemes, table)
+    return int(_lib.load().spade_grouped_workspace_bytes(gs, len(schemes), rows, len(table), d, text_tokens))
+
+
+def grouped_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, schemes, table, text_tokens: int = 0,
+                 out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """table: per head (scheme index, tau, dense)."""
+    heads, d = q.shape[1], q.shape[2]
+    gs, rows = _tables(schemes, table)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        need = int(_lib.load().spade_grouped_workspace_bytes(gs, len(schemes), rows, heads, d, text_tokens))
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    check(_lib.load().spade_grouped_attn(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), gs, len(schemes), rows, heads, d,
+        text_tokens, dtype_code(q.dtype), _dev(workspace, "workspace"), workspace.numel(), _stream(stream)),
+        "spade_grouped_attn")
+    return out
+
+
+def grouped_head_lists(schemes, table, d: int, text_tokens: int, head: int) -> Tuple[int, int]:
+    """Byte offsets of head's (cnt, idx) inside a grouped workspace; (-1, -1) for dense heads."""
+    gs, rows = _tables(schemes, table)
+    co, io = ctypes.c_int64(), ctypes.c_int64()
+    check(_lib.load().spade_grouped_head_lists(gs, len(schemes), rows, len(table), d, text_tokens, head,
+                                               ctypes.byref(co), ctypes.byref(io)), "spade_grouped_head_lists")
+    return co.value, io.value
+
+
+def last_device_status(stream=None) -> int:
+    return int(_lib.load().spade_last_device_status(_stream(stream)))
+
+
+def selftest_bounded_wait(timeout_ns: int, stream=None) -> None:
+    check(_lib.load().spade_selftest_bounded_wait(int(timeout_ns), _stream(stream)),
+          "spade_selftest_bounded_wait")

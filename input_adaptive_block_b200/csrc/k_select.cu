@@ -1,0 +1,246 @@
+// Step 4: the executor's index search, and the cost-ranked work list.
+//
+// SPADE abstract (catalyzex.com): the executor performs a "low-overhead index
+// search"; technical summary (gist.science/paper/2608.03335), Methodology 3,
+// "Flash Block-Sparse Attention": masks are turned into a ranked block-sparse
+// representation for sequential access.
+//
+// Per (head, query block i): keep i, then the other key blocks in descending
+// probability (ties -> lower id) until the kept mass reaches tau.  Instead of
+// sorting, one warp per row finds the cut value by a binary search over the
+// IEEE-754 bit pattern (monotone for non-negative floats): the largest theta
+// with  p_ii + sum_{j != i, p_j >= theta} p_j >= tau.  Blocks above theta are
+// kept, ties at theta are taken lowest id first.  Kept ids are written in
+// ascending order (sequential K/V access); a second kernel ranks the
+// (head, query block) items by cost for the attention scheduler.
+#include "spade_internal.cuh"
+
+namespace spade {
+namespace {
+
+struct SelectTaus {
+  float tau[SPADE_SELECT_MAX_HEADS];
+};
+
+constexpr int kSelWarps = 8;
+
+template <int NPL>
+__global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __restrict__ prob,
+                                                               const __grid_constant__ SelectTaus taus,
+                                                               int* __restrict__ cnt, int* __restrict__ idx,
+                                                               int heads, int nb) {
+  __shared__ float buf[kSelWarps][NPL * 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kSelWarps + warp;
+  if (row >= (long long)heads * nb) return;
+  const int h = (int)(row / nb);
+  const int i = (int)(row - (long long)h * nb);
+  const float* prow = prob + row * nb;
+  float* b = buf[warp];
+  for (int j = lane; j < nb; j += 32) b[j] = prow[j];
+  __syncwarp();
+  const float tau = taus.tau[h];
+  const float diag = b[i];
+  // lane owns j in [lane*NPL, lane*NPL + NPL): contiguous, so ascending output is a lane-order scan
+  float v[NPL];
+#pragma unroll
+  for (int e = 0; e < NPL; ++e) {
+    const int j = lane * NPL + e;
+    v[e] = (j < nb && j != i) ? b[j] : -1.0f;   // -1: never reaches a non-negative threshold
+  }
+  uint32_t keep = 0;   // bit e: element lane*NPL+e kept
+  bool keep_all = tau >= 1.0f;
+  if (!keep_all && diag < tau) {
+    uint32_t u = 0;
+    for (int bit = 29; bit >= 0; --bit) {           // p <= 1 < 2.0f = 0x40000000
+      const uint32_t cand = u | (1u << bit);
+      const float thr = __uint_as_float(cand);
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < NPL; ++e) s += (v[e] >= thr) ? v[e] : 0.f;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (diag + s >= tau) u = cand;
+    }
+    if (u == 0) {
+      keep_all = true;                               // the mass never reaches tau
+    } else {
+      const float theta = __uint_as_float(u);
+      float above = 0.f;
+      int ties = 0;
+#pragma unroll
+      for (int e = 0; e < NPL; ++e) {
+        if (v[e] > theta) { keep |= 1u << e; above += v[e]; }
+        ties += (v[e] == theta);
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        above += __shfl_xor_sync(0xffffffffu, above, o);
+        ties += __shfl_xor_sync(0xffffffffu, ties, o);
+      }
+      if (ties == 1) {
+#pragma unroll
+        for (int e = 0; e < NPL; ++e)
+          if (v[e] == theta) keep |= 1u << e;
+      } else {
+        float mass = diag + above;                   // take tied blocks lowest id first
+        for (int L = 0; L < 32; ++L) {
+          for (int e = 0; e < NPL; ++e) {
+            const bool tie = __shfl_sync(0xffffffffu, v[e] == theta ? 1 : 0, L) != 0;
+            if (tie && mass < tau) {
+              if (lane == L) keep |= 1u << e;
+              mass += theta;
+            }
+          }
+        }
+      }
+    }
+  }
+  if (keep_all) {
+    keep = 0;
+#pragma unroll
+    for (int e = 0; e < NPL; ++e)
+      if (lane * NPL + e < nb) keep |= 1u << e;
+  } else {
+    const int di = i - lane * NPL;                 // the diagonal is always kept
+    if (di >= 0 && di < NPL) keep |= 1u << di;
+  }
+  const int mine = __popc(keep);
+  int pre = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, pre, o);
+    if (lane >= o) pre += t;
+  }
+  const int total = __shfl_sync(0xffffffffu, pre, 31);
+  int* out = idx + row * nb + (pre - mine);
+  int w = 0;
+#pragma unroll
+  for (int e = 0; e < NPL; ++e)
+    if (keep & (1u << e)) out[w++] = lane * NPL + e;
+  if (lane == 0) cnt[row] = total;
+}
+
+// ------------------------------------------------------------ work list --
+// Items (head, query block) ranked by cost = number of key blocks walked,
+// descending (longest first), by a counting sort in one CTA.
+struct WorklistArgs {
+  int heads;
+  int ntb;
+  int n_items;
+  int item_start[SPADE_MAX_HEADS + 1];   // prefix sum of items per head
+  int nb[SPADE_MAX_HEADS];
+  int dense[SPADE_MAX_HEADS];
+  int cnt_off[SPADE_MAX_HEADS];
+};
+
+__device__ __forceinline__ void decode_item(const WorklistArgs& a, int g, int& h, int& qb) {
+  int lo = 0, hi = a.heads - 1;
+  while (lo < hi) {                               // last head with item_start <= g
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.item_start[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  h = lo;
+  qb = g - a.item_start[lo];
+}
+
+__device__ __forceinline__ int item_cost(const WorklistArgs& a, const int* cnt, int h, int qb) {
+  const int nb = a.nb[h];
+  if (a.dense[h] || qb >= nb) return nb + a.ntb;
+  return cnt[a.cnt_off[h] + qb] + a.ntb;
+}
+
+__global__ void __launch_bounds__(1024) worklist_kernel(const __grid_constant__ WorklistArgs a,
+                                                        const int* __restrict__ cnt, int* __restrict__ work) {
+  __shared__ int hist[SPADE_WORKLIST_MAX_COST];
+  __shared__ int warp_tot[32];
+  const int tid = threadIdx.x;
+  for (int i = tid; i < SPADE_WORKLIST_MAX_COST; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  for (int g = tid; g < a.n_items; g += blockDim.x) {
+    int h, qb;
+    decode_item(a, g, h, qb);
+    const int c = min(item_cost(a, cnt, h, qb), SPADE_WORKLIST_MAX_COST - 1);
+    atomicAdd(&hist[SPADE_WORKLIST_MAX_COST - 1 - c], 1);
+  }
+  __syncthreads();
+  // exclusive scan over bins: each thread owns 4 consecutive bins
+  constexpr int PER = SPADE_WORKLIST_MAX_COST / 1024;
+  int local[PER];
+  int s = 0;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) { local[e] = hist[tid * PER + e]; s += local[e]; }
+  const int lane = tid & 31, warp = tid >> 5;
+  int inc = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += t;
+    }
+    warp_tot[lane] = w;
+  }
+  __syncthreads();
+  int base = inc - s + (warp > 0 ? warp_tot[warp - 1] : 0);
+#pragma unroll
+  for (int e = 0; e < PER; ++e) { hist[tid * PER + e] = base; base += local[e]; }
+  __syncthreads();
+  for (int g = tid; g < a.n_items; g += blockDim.x) {
+    int h, qb;
+    decode_item(a, g, h, qb);
+    const int c = min(item_cost(a, cnt, h, qb), SPADE_WORKLIST_MAX_COST - 1);
+    const int pos = atomicAdd(&hist[SPADE_WORKLIST_MAX_COST - 1 - c], 1);
+    work[pos] = (h << 16) | qb;
+  }
+}
+
+template <int NPL>
+cudaError_t launch_select_t(const float* prob, const SelectTaus& t, int* cnt, int* idx, int heads, int nb,
+                            cudaStream_t s) {
+  const long long rows = (long long)heads * nb;
+  const int blocks = (int)((rows + kSelWarps - 1) / kSelWarps);
+  select_kernel<NPL><<<blocks, kSelWarps * 32, 0, s>>>(prob, t, cnt, idx, heads, nb);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_select(const float* prob, const float* tau_host, int* cnt, int* idx, int heads, int nb,
+                          cudaStream_t s) {
+  SelectTaus t;
+  for (int h = 0; h < heads; ++h) t.tau[h] = tau_host[h];
+  const int npl = (nb + 31) / 32;
+  if (npl <= 4) return launch_select_t<4>(prob, t, cnt, idx, heads, nb, s);
+  if (npl <= 8) return launch_select_t<8>(prob, t, cnt, idx, heads, nb, s);
+  if (npl <= 16) return launch_select_t<16>(prob, t, cnt, idx, heads, nb, s);
+  if (npl <= 24) return launch_select_t<24>(prob, t, cnt, idx, heads, nb, s);
+  return launch_select_t<32>(prob, t, cnt, idx, heads, nb, s);
+}
+
+cudaError_t launch_worklist(const AttnArgs& a, cudaStream_t s) {
+  WorklistArgs w;
+  w.heads = a.heads;
+  w.ntb = text_blocks(a.text_tokens);
+  int acc = 0;
+  for (int h = 0; h < a.heads; ++h) {
+    w.item_start[h] = acc;
+    w.nb[h] = a.head[h].nb;
+    w.dense[h] = a.head[h].dense;
+    w.cnt_off[h] = a.head[h].cnt_off;
+    acc += a.head[h].nb + w.ntb;
+  }
+  w.item_start[a.heads] = acc;
+  w.n_items = acc;
+  worklist_kernel<<<1, 1024, 0, s>>>(w, a.cnt, a.work);
+  return cudaGetLastError();
+}
+
+}  // namespace spade

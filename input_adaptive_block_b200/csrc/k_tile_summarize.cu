@@ -1,0 +1,160 @@
+// Step 1 (3D tiling) and step 2 (block-mean Summarizer) of the SPADE executor.
+//
+// SPADE technical summary (gist.science/paper/2608.03335), Methodology 1,
+// "Blocking Scheme Candidates" and "Summarizer & Estimator Expressions";
+// Methodology 3, "Kernel Fusion" (layout transformation fused with
+// summarization).  The summarizer below reads Q/K in token order and reduces
+// each 3D block directly, so the tiled layout is never written on the hot
+// path; the attention kernel gathers its tiles with TMA boxes instead.
+#include "spade_internal.cuh"
+
+namespace spade {
+namespace {
+
+// ---------------------------------------------------------------- tile3d --
+// One CTA per block; each thread moves 16-byte chunks.  Source rows are whole
+// token rows (all heads), so reads are fully coalesced; each (head, slot)
+// destination segment is d*esz contiguous bytes.
+__global__ void tile3d_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict__ xt, Geo g, int heads,
+                              int row_bytes_head) {
+  const int b = blockIdx.x;
+  int t0, y0, x0, et, eh, ew;
+  block_box(g, b, t0, y0, x0, et, eh, ew);
+  const int chunks_head = row_bytes_head / 16;
+  const int chunks_tok = chunks_head * heads;
+  const long long row_bytes = (long long)row_bytes_head * heads;
+  const int total = g.bs * chunks_tok;
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
+    const int slot = i / chunks_tok;
+    const int c = i - slot * chunks_tok;
+    const int h = c / chunks_head;
+    const int cc = c - h * chunks_head;
+    const int xl = slot % g.bw;
+    const int yl = (slot / g.bw) % g.bh;
+    const int tl = slot / (g.bw * g.bh);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (tl < et && yl < eh && xl < ew) {
+      const long long tok = ((long long)(t0 + tl) * g.H + (y0 + yl)) * g.W + (x0 + xl);
+      v = __ldg(reinterpret_cast<const uint4*>(x + tok * row_bytes) + c);
+    }
+    uint8_t* dst = xt + (((long long)h * g.nb + b) * g.bs + slot) * row_bytes_head;
+    reinterpret_cast<uint4*>(dst)[cc] = v;
+  }
+}
+
+// ------------------------------------------------------------- summarize --
+// Work unit = (block b, group of 32 16-byte chunks of a token row restricted
+// to heads [h0, h0+hc)).  One warp per unit; lane l owns chunk 32*group + l
+// and sums it over the block's valid tokens in fp32 (8-token unroll for
+// memory-level parallelism).  Units are dealt round-robin to all warps.
+template <bool BF16>
+__global__ void __launch_bounds__(256) summarize_kernel(const uint8_t* __restrict__ x, float* __restrict__ out,
+                                                         Geo g, long long row_bytes, int head_off_bytes,
+                                                         int chunks, int d) {
+  constexpr int EPC = BF16 ? 8 : 4;  // elements per 16-byte chunk
+  const int lane = threadIdx.x & 31;
+  const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int groups = (chunks + 31) / 32;
+  const long long n_units = (long long)g.nb * groups;
+  for (long long u = gwarp; u < n_units; u += nwarps) {
+    const int b = (int)(u / groups);
+    const int c = (int)(u - (long long)b * groups) * 32 + lane;
+    int t0, y0, x0, et, eh, ew;
+    block_box(g, b, t0, y0, x0, et, eh, ew);
+    const int nvalid = et * eh * ew;
+    float acc[EPC];
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+    if (c < chunks) {
+      const uint8_t* base = x + head_off_bytes + (long long)c * 16;
+      int i = 0;
+      for (; i + 8 <= nvalid; i += 8) {
+        uint4 v[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int ii = i + r;
+          const int xl = ii % ew, yl = (ii / ew) % eh, tl = ii / (ew * eh);
+          const long long tok = ((long long)(t0 + tl) * g.H + (y0 + yl)) * g.W + (x0 + xl);
+          v[r] = __ldg(reinterpret_cast<const uint4*>(base + tok * row_bytes));
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          if (BF16) {
+            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[r]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float2 f = __bfloat1622float2(p[e]);
+              acc[2 * e] += f.x;
+              acc[2 * e + 1] += f.y;
+            }
+          } else {
+            const float* f = reinterpret_cast<const float*>(&v[r]);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+          }
+        }
+      }
+      for (; i < nvalid; ++i) {
+        const int xl = i % ew, yl = (i / ew) % eh, tl = i / (ew * eh);
+        const long long tok = ((long long)(t0 + tl) * g.H + (y0 + yl)) * g.W + (x0 + xl);
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(base + tok * row_bytes));
+        if (BF16) {
+          const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(p[e]);
+            acc[2 * e] += f.x;
+            acc[2 * e + 1] += f.y;
+          }
+        } else {
+          const float* f = reinterpret_cast<const float*>(&v);
+#pragma unroll
+          for (int e = 0; e < EPC; ++e) acc[e] += f[e];
+        }
+      }
+      const float inv = 1.0f / (float)nvalid;
+      const int e0 = c * EPC;             // element index within the head-range row
+      const int h = e0 / d, dd = e0 - h * d;
+      float* o = out + ((long long)h * g.nb + b) * d + dd;
+      if (BF16) {
+        reinterpret_cast<float4*>(o)[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        reinterpret_cast<float4*>(o)[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+      } else {
+        reinterpret_cast<float4*>(o)[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_tile3d(const void* x, void* xt, const Geo& g, int heads, int d, spade_dtype dt,
+                          cudaStream_t s) {
+  const int esz = dt == SPADE_BF16 ? 2 : 4;
+  tile3d_kernel<<<g.nb, 256, 0, s>>>(static_cast<const uint8_t*>(x), static_cast<uint8_t*>(xt), g, heads,
+                                     d * esz);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_summarize(const void* x, float* out, const Geo& g, int heads_total, int h0, int hc, int d,
+                             spade_dtype dt, cudaStream_t s) {
+  const int esz = dt == SPADE_BF16 ? 2 : 4;
+  const long long row_bytes = (long long)heads_total * d * esz;
+  const int chunks = hc * d * esz / 16;
+  const int groups = (chunks + 31) / 32;
+  const long long units = (long long)g.nb * groups;
+  long long blocks = (units + 7) / 8;                  // 8 warps per CTA
+  const long long cap = 2LL * num_sms();               // 16 resident warps per SM
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  if (dt == SPADE_BF16)
+    summarize_kernel<true><<<(int)blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), out, g, row_bytes,
+                                                        h0 * d * esz, chunks, d);
+  else
+    summarize_kernel<false><<<(int)blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), out, g, row_bytes,
+                                                         h0 * d * esz, chunks, d);
+  return cudaGetLastError();
+}
+
+}  // namespace spade

@@ -1,0 +1,403 @@
+// C ABI of the SPADE executor hot path (declared in include/spade.h):
+// argument validation, workspace layout, and the order of launches for the
+// single steps and for the grouped (mixed-scheme) layer.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "spade_internal.cuh"
+
+// Latched device status (SPADE_OK / SPADE_ERR_TIMEOUT), one per device.
+__device__ int g_spade_status;
+
+namespace spade {
+
+namespace {
+
+thread_local std::string g_err;
+
+spade_status fail(spade_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+spade_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(SPADE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+int* status_ptr() {
+  static int* ptrs[kMaxDevices] = {nullptr};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_spade_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+spade_status check_geom(const spade_geom& g) {
+  if (g.T <= 0 || g.H <= 0 || g.W <= 0 || g.bt <= 0 || g.bh <= 0 || g.bw <= 0)
+    return fail(SPADE_ERR_INVALID, "geometry has a non-positive extent");
+  if (g.bt > 256 || g.bh > 256 || g.bw > 256) return fail(SPADE_ERR_UNSUPPORTED, "block extent above 256");
+  const long long bs = (long long)g.bt * g.bh * g.bw;
+  if (bs > 1024) return fail(SPADE_ERR_UNSUPPORTED, "block size %lld above 1024", bs);
+  const Geo gg = make_geo(g);
+  if (gg.nb > 65535) return fail(SPADE_ERR_UNSUPPORTED, "more than 65535 blocks");
+  return SPADE_OK;
+}
+
+spade_status check_d_dt(int d, spade_dtype dt) {
+  if (d != 64 && d != 128) return fail(SPADE_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", d);
+  if (dt != SPADE_F32 && dt != SPADE_BF16) return fail(SPADE_ERR_INVALID, "unknown dtype %d", (int)dt);
+  return SPADE_OK;
+}
+
+cudaStream_t as_cuda(spade_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Layout of the grouped workspace (byte offsets).
+struct GroupLayout {
+  int n_sparse[SPADE_MAX_SCHEMES];
+  std::vector<int> heads_of[SPADE_MAX_SCHEMES];   // sparse heads per scheme, ascending
+  size_t qmean[SPADE_MAX_SCHEMES], kmean[SPADE_MAX_SCHEMES], prob[SPADE_MAX_SCHEMES];
+  size_t cnt[SPADE_MAX_SCHEMES], idx[SPADE_MAX_SCHEMES];
+  std::vector<int> pos;                             // position of head h in its scheme group
+  size_t work;
+  int n_items;
+  size_t total;
+};
+
+spade_status plan_group(const spade_geom* schemes, int n_schemes, const spade_head_scheme* table, int heads,
+                        int d, int text_tokens, GroupLayout& L) {
+  if (!schemes || !table) return fail(SPADE_ERR_INVALID, "null scheme table");
+  if (n_schemes < 1 || n_schemes > SPADE_MAX_SCHEMES)
+    return fail(SPADE_ERR_UNSUPPORTED, "n_schemes=%d (1..%d)", n_schemes, SPADE_MAX_SCHEMES);
+  if (heads < 1 || heads > SPADE_MAX_HEADS) return fail(SPADE_ERR_UNSUPPORTED, "heads=%d (1..128)", heads);
+  if (text_tokens < 0) return fail(SPADE_ERR_INVALID, "negative text_tokens");
+  if (d != 64 && d != 128) return fail(SPADE_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", d);
+  const long long N = (long long)schemes[0].T * schemes[0].H * schemes[0].W;
+  for (int s = 0; s < n_schemes; ++s) {
+    spade_status st = check_geom(schemes[s]);
+    if (st != SPADE_OK) return st;
+    if ((long long)schemes[s].T * schemes[s].H * schemes[s].W != N)
+      return fail(SPADE_ERR_INVALID, "scheme %d covers a different number of tokens", s);
+  }
+  L.pos.assign(heads, -1);
+  for (int s = 0; s < n_schemes; ++s) { L.n_sparse[s] = 0; L.heads_of[s].clear(); }
+  for (int h = 0; h < heads; ++h) {
+    const spade_head_scheme& r = table[h];
+    if (r.scheme < 0 || r.scheme >= n_schemes) return fail(SPADE_ERR_INVALID, "head %d: scheme %d", h, r.scheme);
+    if (r.dense != 0 && r.dense != 1) return fail(SPADE_ERR_INVALID, "head %d: dense flag %d", h, r.dense);
+    if (!r.dense && !(r.tau > 0.f && r.tau <= 1e30f)) return fail(SPADE_ERR_INVALID, "head %d: tau", h);
+    if (!r.dense) {
+      L.pos[h] = L.n_sparse[r.scheme]++;
+      L.heads_of[r.scheme].push_back(h);
+    }
+  }
+  size_t off = 0;
+  const int ntb = text_blocks(text_tokens);
+  L.n_items = 0;
+  for (int h = 0; h < heads; ++h) L.n_items += make_geo(schemes[table[h].scheme]).nb + ntb;
+  for (int s = 0; s < n_schemes; ++s) {
+    const Geo g = make_geo(schemes[s]);
+    const size_t hs = L.n_sparse[s];
+    if (hs > 0) {
+      if (g.nb > SPADE_SELECT_MAX_NB) return fail(SPADE_ERR_UNSUPPORTED, "scheme %d: nb=%d above 1024", s, g.nb);
+    }
+    L.qmean[s] = off; off = align256(off + hs * g.nb * d * sizeof(float));
+    L.kmean[s] = off; off = align256(off + hs * g.nb * d * sizeof(float));
+    L.prob[s] = off;  off = align256(off + hs * g.nb * g.nb * sizeof(float));
+    L.cnt[s] = off;   off = align256(off + hs * g.nb * sizeof(int));
+    L.idx[s] = off;   off = align256(off + hs * g.nb * g.nb * sizeof(int));
+  }
+  L.work = off;
+  off = align256(off + (size_t)L.n_items * sizeof(int));
+  L.total = off;
+  return SPADE_OK;
+}
+
+spade_status run_attention(AttnArgs& a, cudaStream_t s) {
+  a.status = status_ptr();
+  if (!a.status) return fail(SPADE_ERR_CUDA, "device status word unavailable");
+  cudaError_t e = launch_worklist(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "work list");
+  if (attn_tc_supported(a)) {
+    const char* why = "";
+    e = launch_attn_tc(a, s, &why);
+    if (e != cudaSuccess) return fail(SPADE_ERR_CUDA, "tensor-core attention: %s (%s)", cudaGetErrorString(e), why);
+  } else {
+    for (int sc = 0; sc < a.n_schemes; ++sc)
+      if (a.geo[sc].bs > 128) return fail(SPADE_ERR_UNSUPPORTED, "CUDA-core attention needs blocks <= 128 slots");
+    e = launch_attn_simt(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "CUDA-core attention");
+  }
+  return SPADE_OK;
+}
+
+}  // namespace
+
+int num_sms() {
+  static int sms[kMaxDevices] = {0};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 1;
+  if (!sms[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    sms[dev] = v > 0 ? v : 1;
+  }
+  return sms[dev];
+}
+
+long long device_wait_timeout_ns() {
+  static long long ns = -1;
+  if (ns < 0) {
+    const char* e = getenv("SPADE_WAIT_TIMEOUT_MS");
+    long long ms = e ? atoll(e) : 10000;
+    if (ms <= 0) ms = 10000;
+    ns = ms * 1000000LL;
+  }
+  return ns;
+}
+
+}  // namespace spade
+
+using namespace spade;
+
+extern "C" {
+
+int spade_version(void) { return 1; }
+
+const char* spade_status_string(spade_status s) {
+  switch (s) {
+    case SPADE_OK: return "ok";
+    case SPADE_ERR_INVALID: return "invalid argument";
+    case SPADE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SPADE_ERR_CUDA: return "CUDA error";
+    case SPADE_ERR_TIMEOUT: return "device wait timed out";
+    case SPADE_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char* spade_last_error_message(void) { return g_err.c_str(); }
+
+spade_status spade_tile3d(const void* x, void* xt, spade_geom g, int heads, int d, spade_dtype dt,
+                          spade_stream_t stream) {
+  spade_status st = check_geom(g);
+  if (st != SPADE_OK) return st;
+  if ((st = check_d_dt(d, dt)) != SPADE_OK) return st;
+  if (!x || !xt) return fail(SPADE_ERR_INVALID, "null pointer");
+  if (!aligned16(x) || !aligned16(xt)) return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  if (heads < 1) return fail(SPADE_ERR_INVALID, "heads=%d", heads);
+  cudaError_t e = launch_tile3d(x, xt, make_geo(g), heads, d, dt, as_cuda(stream));
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "tile3d");
+}
+
+spade_status spade_summarize(const void* x, float* xmean, spade_geom g, int heads, int d, spade_dtype dt,
+                             spade_stream_t stream) {
+  spade_status st = check_geom(g);
+  if (st != SPADE_OK) return st;
+  if ((st = check_d_dt(d, dt)) != SPADE_OK) return st;
+  if (!x || !xmean) return fail(SPADE_ERR_INVALID, "null pointer");
+  if (!aligned16(x) || !aligned16(xmean)) return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  if (heads < 1) return fail(SPADE_ERR_INVALID, "heads=%d", heads);
+  cudaError_t e = launch_summarize(x, xmean, make_geo(g), heads, 0, heads, d, dt, as_cuda(stream));
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "summarize");
+}
+
+spade_status spade_estimate(const float* qmean, const float* kmean, float* prob, int heads, int nb, int d,
+                            spade_stream_t stream) {
+  if (!qmean || !kmean || !prob) return fail(SPADE_ERR_INVALID, "null pointer");
+  if (!aligned16(qmean) || !aligned16(kmean) || !aligned16(prob))
+    return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  if (heads < 1 || heads > 65535) return fail(SPADE_ERR_INVALID, "heads=%d", heads);
+  if (nb < 1) return fail(SPADE_ERR_INVALID, "nb=%d", nb);
+  if (nb > SPADE_ESTIMATE_MAX_NB) return fail(SPADE_ERR_UNSUPPORTED, "nb=%d above %d", nb, SPADE_ESTIMATE_MAX_NB);
+  if (d != 64 && d != 128) return fail(SPADE_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", d);
+  cudaError_t e = launch_estimate(qmean, kmean, prob, heads, nb, d, as_cuda(stream));
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "estimate");
+}
+
+spade_status spade_select(const float* prob, const float* tau_host, int* cnt, int* idx, int heads, int nb,
+                          spade_stream_t stream) {
+  if (!prob || !tau_host || !cnt || !idx) return fail(SPADE_ERR_INVALID, "null pointer");
+  if (heads < 1 || heads > SPADE_SELECT_MAX_HEADS) return fail(SPADE_ERR_UNSUPPORTED, "heads=%d (1..1024)", heads);
+  if (nb < 1) return fail(SPADE_ERR_INVALID, "nb=%d", nb);
+  if (nb > SPADE_SELECT_MAX_NB) return fail(SPADE_ERR_UNSUPPORTED, "nb=%d above %d", nb, SPADE_SELECT_MAX_NB);
+  for (int h = 0; h < heads; ++h)
+    if (!(tau_host[h] > 0.f && tau_host[h] <= 1e30f)) return fail(SPADE_ERR_INVALID, "tau[%d] must be > 0", h);
+  cudaError_t e = launch_select(prob, tau_host, cnt, idx, heads, nb, as_cuda(stream));
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "select");
+}
+
+size_t spade_attn_workspace_bytes(spade_geom g, int heads, int d, int text_tokens) {
+  (void)d;
+  if (heads < 1 || text_tokens < 0 || g.bt <= 0 || g.bh <= 0 || g.bw <= 0 || g.T <= 0 || g.H <= 0 || g.W <= 0)
+    return 0;
+  const Geo gg = make_geo(g);
+  return align256((size_t)heads * (gg.nb + text_blocks(text_tokens)) * sizeof(int));
+}
+
+spade_status spade_block_sparse_attn(const void* q, const void* k, const void* v, void* out, const int* cnt,
+                                     const int* idx, spade_geom g, int heads, int d, int text_tokens,
+                                     spade_dtype dt, void* workspace, size_t ws_bytes, spade_stream_t stream) {
+  spade_status st = check_geom(g);
+  if (st != SPADE_OK) return st;
+  if ((st = check_d_dt(d, dt)) != SPADE_OK) return st;
+  if (!q || !k || !v || !out) return fail(SPADE_ERR_INVALID, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  if ((cnt == nullptr) != (idx == nullptr)) return fail(SPADE_ERR_INVALID, "cnt and idx must both be set or both NULL");
+  if (heads < 1 || heads > SPADE_MAX_HEADS) return fail(SPADE_ERR_UNSUPPORTED, "heads=%d (1..128)", heads);
+  if (text_tokens < 0) return fail(SPADE_ERR_INVALID, "negative text_tokens");
+  const size_t need = spade_attn_workspace_bytes(g, heads, d, text_tokens);
+  if (!workspace || ws_bytes < need) return fail(SPADE_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out;
+  a.n_schemes = 1;
+  a.geo[0] = make_geo(g);
+  a.heads = heads; a.d = d; a.text_tokens = text_tokens; a.N = g.T * g.H * g.W; a.dt = dt;
+  const int nb = a.geo[0].nb;
+  for (int h = 0; h < heads; ++h) {
+    a.head[h].scheme = 0;
+    a.head[h].nb = nb;
+    a.head[h].dense = cnt == nullptr;
+    a.head[h].cnt_off = h * nb;
+    a.head[h].idx_off = (long long)h * nb * nb;
+  }
+  a.cnt = cnt; a.idx = idx;
+  a.work = static_cast<int*>(workspace);
+  a.n_items = heads * (nb + text_blocks(text_tokens));
+  return run_attention(a, as_cuda(stream));
+}
+
+size_t spade_grouped_workspace_bytes(const spade_geom* schemes, int n_schemes, const spade_head_scheme* table,
+                                     int heads, int d, int text_tokens) {
+  GroupLayout L;
+  if (plan_group(schemes, n_schemes, table, heads, d, text_tokens, L) != SPADE_OK) return 0;
+  return L.total;
+}
+
+spade_status spade_grouped_head_lists(const spade_geom* schemes, int n_schemes, const spade_head_scheme* table,
+                                      int heads, int d, int text_tokens, int head, int64_t* cnt_offset,
+                                      int64_t* idx_offset) {
+  GroupLayout L;
+  spade_status st = plan_group(schemes, n_schemes, table, heads, d, text_tokens, L);
+  if (st != SPADE_OK) return st;
+  if (head < 0 || head >= heads || !cnt_offset || !idx_offset) return fail(SPADE_ERR_INVALID, "head/outputs");
+  if (table[head].dense) { *cnt_offset = -1; *idx_offset = -1; return SPADE_OK; }
+  const int s = table[head].scheme;
+  const Geo g = make_geo(schemes[s]);
+  *cnt_offset = (int64_t)(L.cnt[s] + (size_t)L.pos[head] * g.nb * sizeof(int));
+  *idx_offset = (int64_t)(L.idx[s] + (size_t)L.pos[head] * g.nb * g.nb * sizeof(int));
+  return SPADE_OK;
+}
+
+spade_status spade_grouped_attn(const void* q, const void* k, const void* v, void* out, const spade_geom* schemes,
+                                int n_schemes, const spade_head_scheme* table, int heads, int d, int text_tokens,
+                                spade_dtype dt, void* workspace, size_t ws_bytes, spade_stream_t stream) {
+  GroupLayout L;
+  spade_status st = plan_group(schemes, n_schemes, table, heads, d, text_tokens, L);
+  if (st != SPADE_OK) return st;
+  if ((st = check_d_dt(d, dt)) != SPADE_OK) return st;
+  if (!q || !k || !v || !out) return fail(SPADE_ERR_INVALID, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+    return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  if (!workspace || ws_bytes < L.total) return fail(SPADE_ERR_WORKSPACE, "workspace needs %zu bytes", L.total);
+  cudaStream_t s = as_cuda(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int N = schemes[0].T * schemes[0].H * schemes[0].W;
+  // steps 1-4 per scheme, for its non-dense heads
+  for (int sc = 0; sc < n_schemes; ++sc) {
+    const int hs = L.n_sparse[sc];
+    if (hs == 0) continue;
+    const Geo g = make_geo(schemes[sc]);
+    float* qm = reinterpret_cast<float*>(ws + L.qmean[sc]);
+    float* km = reinterpret_cast<float*>(ws + L.kmean[sc]);
+    const std::vector<int>& hl = L.heads_of[sc];
+    for (int i = 0; i < hs;) {                        // contiguous runs of heads
+      int j = i + 1;
+      while (j < hs && hl[j] == hl[j - 1] + 1) ++j;
+      const size_t o = (size_t)i * g.nb * d;
+      cudaError_t e = launch_summarize(q, qm + o, g, heads, hl[i], j - i, d, dt, s);
+      if (e == cudaSuccess) e = launch_summarize(k, km + o, g, heads, hl[i], j - i, d, dt, s);
+      if (e != cudaSuccess) return cuda_fail(e, "summarize");
+      i = j;
+    }
+    float* prob = reinterpret_cast<float*>(ws + L.prob[sc]);
+    cudaError_t e = launch_estimate(qm, km, prob, hs, g.nb, d, s);
+    if (e != cudaSuccess) return cuda_fail(e, "estimate");
+    std::vector<float> taus(hs);
+    for (int i = 0; i < hs; ++i) taus[i] = table[hl[i]].tau;
+    e = launch_select(prob, taus.data(), reinterpret_cast<int*>(ws + L.cnt[sc]),
+                      reinterpret_cast<int*>(ws + L.idx[sc]), hs, g.nb, s);
+    if (e != cudaSuccess) return cuda_fail(e, "select");
+  }
+  // step 5: one grouped launch over every head
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out;
+  a.n_schemes = n_schemes;
+  for (int sc = 0; sc < n_schemes; ++sc) a.geo[sc] = make_geo(schemes[sc]);
+  a.heads = heads; a.d = d; a.text_tokens = text_tokens; a.N = N; a.dt = dt;
+  for (int h = 0; h < heads; ++h) {
+    const int sc = table[h].scheme;
+    const Geo& g = a.geo[sc];
+    a.head[h].scheme = sc;
+    a.head[h].nb = g.nb;
+    a.head[h].dense = table[h].dense;
+    if (!table[h].dense) {
+      a.head[h].cnt_off = (int)((L.cnt[sc] + (size_t)L.pos[h] * g.nb * sizeof(int)) / sizeof(int));
+      a.head[h].idx_off = (long long)((L.idx[sc] + (size_t)L.pos[h] * g.nb * g.nb * sizeof(int)) / sizeof(int));
+    }
+  }
+  a.cnt = reinterpret_cast<const int*>(ws);
+  a.idx = reinterpret_cast<const int*>(ws);
+  a.work = reinterpret_cast<int*>(ws + L.work);
+  a.n_items = L.n_items;
+  return run_attention(a, s);
+}
+
+spade_status spade_last_device_status(spade_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(as_cuda(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_spade_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_spade_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
+  return static_cast<spade_status>(v);
+}
+
+spade_status spade_selftest_bounded_wait(int64_t timeout_ns, spade_stream_t stream) {
+  if (timeout_ns <= 0 || timeout_ns > 10000000000LL) return fail(SPADE_ERR_INVALID, "timeout_ns out of range");
+  int* sp = status_ptr();
+  if (!sp) return fail(SPADE_ERR_CUDA, "device status word unavailable");
+  cudaError_t e = launch_bounded_wait_selftest(sp, timeout_ns, as_cuda(stream));
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "bounded-wait self test");
+}
+
+}  // extern "C"

@@ -17,3 +17,6 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return GOLDEN
+
+# bounded device waits give up after 2 s in tests (the library default is 10 s)
+os.environ.setdefault("SPADE_WAIT_TIMEOUT_MS", "2000")

@@ -1,0 +1,108 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every entry
+point include/spade.h declares, and rejects bad arguments on the host before
+any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from input_adaptive_block_b200 import _lib
+from input_adaptive_block_b200._lib import SpadeGeom, SpadeHeadScheme
+from spade_workloads import CONFIGS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "spade.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(spade_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = _declared()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, n
+    assert lib.spade_version() == 1
+
+
+def test_status_strings():
+    lib = _lib.load()
+    for s in range(6):
+        assert lib.spade_status_string(s)
+    assert lib.spade_status_string(99) == b"unknown status"
+
+
+def _mixed_tables():
+    wl = CONFIGS["mixed"]
+    gs = (SpadeGeom * len(wl.schemes))(*[SpadeGeom(*s.as_tuple()) for s in wl.schemes])
+    rows = (SpadeHeadScheme * wl.heads)(*[SpadeHeadScheme(sc, t, int(dn)) for sc, t, dn in
+                                          zip(wl.head_scheme, wl.head_tau, wl.head_dense)])
+    return wl, gs, rows
+
+
+def test_grouped_workspace_layout_host_only():
+    lib = _lib.load()
+    wl, gs, rows = _mixed_tables()
+    total = lib.spade_grouped_workspace_bytes(gs, 3, rows, wl.heads, wl.d, 0)
+    # lower bound: the per-scheme arrays of the sparse heads plus the work list
+    lower = 0
+    for s_id, sc in enumerate(wl.schemes):
+        hs = sum(1 for h in range(wl.heads) if wl.head_scheme[h] == s_id and not wl.head_dense[h])
+        lower += hs * sc.nb * (2 * wl.d * 4 + 2 * sc.nb * 4 + 4)
+    n_items = sum(wl.schemes[wl.head_scheme[h]].nb for h in range(wl.heads))
+    lower += 4 * n_items
+    assert lower <= total <= lower + 64 * 256
+    # head lists: dense heads have none; sparse heads get distinct, ordered regions
+    co, io = ctypes.c_int64(), ctypes.c_int64()
+    assert lib.spade_grouped_head_lists(gs, 3, rows, wl.heads, wl.d, 0, 0, ctypes.byref(co), ctypes.byref(io)) == 0
+    assert co.value == -1 and io.value == -1
+    prev = -1
+    for h in range(13, 27):
+        assert lib.spade_grouped_head_lists(gs, 3, rows, wl.heads, wl.d, 0, h,
+                                            ctypes.byref(co), ctypes.byref(io)) == 0
+        assert co.value > prev and io.value % 4 == 0 and io.value + 630 * 630 * 4 <= total
+        prev = co.value
+
+
+def test_host_validation_errors():
+    lib = _lib.load()
+    wl, gs, rows = _mixed_tables()
+    # bad scheme index, bad tau, too many schemes, bad d
+    bad = (SpadeHeadScheme * 2)(SpadeHeadScheme(5, 0.9, 0), SpadeHeadScheme(0, 0.9, 0))
+    assert lib.spade_grouped_workspace_bytes(gs, 3, bad, 2, 128, 0) == 0
+    bad = (SpadeHeadScheme * 1)(SpadeHeadScheme(1, -0.5, 0))
+    assert lib.spade_grouped_workspace_bytes(gs, 3, bad, 1, 128, 0) == 0
+    assert lib.spade_grouped_workspace_bytes(gs, 5, rows, wl.heads, 128, 0) == 0
+    assert lib.spade_grouped_workspace_bytes(gs, 3, rows, wl.heads, 96, 0) == 0
+    g = SpadeGeom(21, 45, 80, 2, 8, 8)
+    fake = ctypes.c_void_p(1 << 20)                 # never dereferenced: validation fails first
+    taus = (ctypes.c_float * 1)(0.9)
+    assert lib.spade_select(fake, taus, fake, fake, 1, 2000, None) == _lib.SPADE_ERR_UNSUPPORTED
+    assert lib.spade_select(None, taus, fake, fake, 1, 10, None) == _lib.SPADE_ERR_INVALID
+    bad_tau = (ctypes.c_float * 1)(0.0)
+    assert lib.spade_select(fake, bad_tau, fake, fake, 1, 10, None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_estimate(fake, fake, fake, 1, 4096, 128, None) == _lib.SPADE_ERR_UNSUPPORTED
+    assert lib.spade_block_sparse_attn(fake, fake, fake, fake, None, None, g, 40, 96, 0, 1, fake, 1 << 20,
+                                       None) == _lib.SPADE_ERR_UNSUPPORTED
+    assert lib.spade_block_sparse_attn(fake, fake, fake, fake, None, None, g, 40, 128, 0, 1, fake, 16,
+                                       None) == _lib.SPADE_ERR_WORKSPACE
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.spade_block_sparse_attn(odd, fake, fake, fake, None, None, g, 40, 128, 0, 1, fake, 1 << 20,
+                                       None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_block_sparse_attn(fake, fake, fake, fake, fake, None, g, 40, 128, 0, 1, fake, 1 << 20,
+                                       None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_tile3d(fake, fake, SpadeGeom(0, 1, 1, 1, 1, 1), 1, 128, 1, None) == _lib.SPADE_ERR_INVALID
+    assert b"extent" in lib.spade_last_error_message()
+
+
+def test_attn_workspace_bytes():
+    lib = _lib.load()
+    g = SpadeGeom(21, 45, 80, 2, 8, 8)
+    assert lib.spade_attn_workspace_bytes(g, 40, 128, 0) >= 40 * 660 * 4
+    assert lib.spade_attn_workspace_bytes(g, 40, 128, 256) >= 40 * 662 * 4
+    assert lib.spade_attn_workspace_bytes(SpadeGeom(0, 1, 1, 1, 1, 1), 1, 128, 0) == 0
