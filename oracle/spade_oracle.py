@@ -175,13 +175,24 @@ def select(P: np.ndarray, taus: Sequence[float]) -> Tuple[np.ndarray, np.ndarray
 
 
 def selection_margin(p: np.ndarray, i: int, tau: float) -> float:
-    """How far row i is from changing its kept set, in probability units:
-    min(p_last_kept - p_first_dropped, tau - mass_before_last, mass_after_last - tau).
-    Rows with a small margin may legitimately differ between fp32 and fp64."""
+    """How far row i is from changing its kept set, in the estimator's score
+    units (pooled logits; a probability ratio p_a/p_b is a score difference
+    ln(p_a/p_b)).  It is the smallest of
+      * ln(p_last_kept / p_first_dropped): the score gap at the cut;
+      * (tau - C_before_last) / (C (1 - C)) and (C_after_last - tau) / (C (1 - C)):
+        the mass slack on either side of tau divided by its first-order
+        sensitivity to a shift of the kept blocks' scores against the rest
+        (d C / d shift = C (1 - C) for a softmax).
+    Rows whose margin is small may legitimately differ between a float32 and
+    a float64 evaluation; rows above the threshold may not."""
     nb = len(p)
     if tau >= 1.0:
         return math.inf
     others = sorted((j for j in range(nb) if j != i), key=lambda j: (-p[j], j))
+
+    def sens(c):
+        return max(c * (1.0 - c), 1e-300)
+
     mass = float(p[i])
     k = 0
     prev = None
@@ -190,12 +201,13 @@ def selection_margin(p: np.ndarray, i: int, tau: float) -> float:
         mass += float(p[others[k]])
         k += 1
     if mass < tau:            # every block kept because the mass never reached tau
-        return tau - mass
+        return 0.0
     if k == 0:                # the diagonal alone reached tau
-        return mass - tau
-    m = min(tau - prev, mass - tau)
+        return (mass - tau) / sens(mass)
+    m = min((tau - prev) / sens(prev), (mass - tau) / sens(mass))
     if k < len(others):
-        m = min(m, float(p[others[k - 1]] - p[others[k]]))
+        a, b = float(p[others[k - 1]]), float(p[others[k]])
+        m = min(m, math.log(a / b) if b > 0.0 else math.inf)
     return m
 
 

@@ -3,6 +3,8 @@ masks, and compare with the oracle under the tolerances of the method's
 precision (bf16 inputs, fp32 accumulation)."""
 from __future__ import annotations
 
+import math
+
 import numpy as np
 import torch
 
@@ -63,13 +65,44 @@ def oracle_selection(wl: Workload, qh: np.ndarray, kh: np.ndarray, h: int):
     return P, kept, margins
 
 
-def compare_kept(gpu_kept, ora_kept, margins, thr=MARGIN):
-    """Bit-exact on rows whose oracle margin exceeds thr; returns
-    (checked, mismatched_rows, skipped) and asserts every GPU row is a valid
-    ascending, diagonal-containing list."""
+def valid_cut(p: np.ndarray, i: int, tau: float, kept, mass_tol: float = 1e-4,
+              score_tol: float = 1e-3) -> bool:
+    """Property every kept list must have, in the oracle's fp64 probabilities,
+    whatever its margin: it contains i, reaches tau (up to mass_tol), is
+    minimal (dropping its smallest non-diagonal block falls below tau), and no
+    dropped block scores above a kept one by more than score_tol."""
+    kept = list(kept)
+    nb = len(p)
+    if i not in kept:
+        return False
+    if tau >= 1.0 or len(kept) == nb:
+        return len(kept) == nb or float(np.sum(p[kept])) >= tau - mass_tol
+    mass = float(np.sum(p[kept]))
+    if mass < tau - mass_tol:
+        return False
+    others = [j for j in kept if j != i]
+    if not others:
+        return True
+    low = min(float(p[j]) for j in others)
+    if mass - low >= tau + mass_tol:
+        return False
+    dropped = np.setdiff1d(np.arange(nb), kept)
+    if len(dropped) and low > 0:
+        if math.log(float(p[dropped].max()) / low) > score_tol:
+            return False
+    return True
+
+
+def compare_kept(gpu_kept, ora_kept, margins, thr=MARGIN, P=None, tau=None):
+    """Bit-exact on rows whose oracle margin (score units) exceeds thr; every
+    row must be ascending, contain its diagonal and, when the oracle's
+    probabilities P are given, pass valid_cut.  Returns
+    (checked, mismatched_rows, skipped)."""
     checked, bad, skipped = 0, [], 0
     for i, (g, o) in enumerate(zip(gpu_kept, ora_kept)):
         assert g == sorted(set(g)) and i in g and all(0 <= j < len(gpu_kept) for j in g), (i, g)
+        if P is not None:
+            assert valid_cut(P[i], i, tau, g), (i, g, o)
         if margins[i] > thr:
             checked += 1
             if g != o:

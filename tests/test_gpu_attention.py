@@ -71,8 +71,8 @@ def test_grouped_layer_parity(wl):
     for h in range(wl.heads):
         if wl.head_dense[h]:
             continue
-        _, ok, mg = oracle_selection(wl, qn[:, h: h + 1], kn[:, h: h + 1], h)
-        _, bad, _ = compare_kept(kept(h), ok, mg)
+        P, ok, mg = oracle_selection(wl, qn[:, h: h + 1], kn[:, h: h + 1], h)
+        _, bad, _ = compare_kept(kept(h), ok, mg, P=P, tau=wl.head_tau[h])
         assert not bad, (h, bad[:5])
 
 

@@ -84,10 +84,10 @@ def test_select_against_oracle_chain(wl):
         gk = [list(idx[h, i, : cnt[h, i]]) for i in range(nb)]
         ok = [O.select_row(Pref[h, i], i, wl.head_tau[h]) for i in range(nb)]
         mg = [O.selection_margin(Pref[h, i], i, wl.head_tau[h]) for i in range(nb)]
-        checked, bad, _ = compare_kept(gk, ok, mg)
+        checked, bad, _ = compare_kept(gk, ok, mg, P=Pref[h], tau=wl.head_tau[h])
         assert not bad, (h, bad[:5])
         total_checked += checked
-    assert total_checked >= 0.9 * wl.heads * Pref.shape[1] or Pref.shape[1] < 4
+    assert total_checked >= 0.5 * wl.heads * Pref.shape[1]
 
 
 @pytest.mark.parametrize("nb", [5, 33, 100, 660, 1020, 1024])
@@ -112,7 +112,7 @@ def test_select_random_rows(nb, tau):
                 assert gk[i] == sorted([i] + others[: int(cnt[h, i]) - 1]), i
                 assert abs(int(cnt[h, i]) - len(ok[i])) <= 1, i
             continue
-        _, bad, _ = compare_kept(gk, ok, mg)
+        _, bad, _ = compare_kept(gk, ok, mg, P=Pn[h], tau=tau)
         assert not bad, (h, bad[:5])
 
 
