@@ -124,8 +124,9 @@ spade_status spade_select(const float* prob, const float* tau_host, int* cnt, in
  * cnt,idx : from spade_select for this scheme ([heads, nb], [heads, nb, nb]);
  *           cnt == NULL means every head is dense.
  * workspace: device scratch of spade_attn_workspace_bytes() bytes (work list).
- * Paths: bf16 with BS == 128 and d in {64,128} runs the tcgen05/TMEM/TMA
- * kernel; everything else (fp32, other block sizes) the CUDA-core kernel. */
+ * Paths: bf16 with BS == 128, d in {64,128} and nb + ceil(text_tokens/128)
+ * <= 1280 runs the tcgen05/TMEM/TMA kernel; everything else (fp32, other
+ * block sizes, longer lists) the CUDA-core kernel (blocks of <= 128 slots). */
 size_t spade_attn_workspace_bytes(spade_geom g, int heads, int d, int text_tokens);
 spade_status spade_block_sparse_attn(const void* q, const void* k, const void* v, void* out,
                                      const int* cnt, const int* idx, spade_geom g,
@@ -170,6 +171,12 @@ int spade_version(void);
  * timeout_ns; the device status must then read SPADE_ERR_TIMEOUT.  Exercises
  * the bounded-wait error path without faulting or hanging the GPU. */
 spade_status spade_selftest_bounded_wait(int64_t timeout_ns, spade_stream_t stream);
+
+/* Evaluates, for n device floats x (x <= 8), the polynomial 2^x the attention
+ * kernel uses for part of its softmax exponentials (round-to-nearest range
+ * reduction, cubic on [-1/2, 1/2]; relative error <= 1e-4 for x >= -125,
+ * inputs below -125 are clamped).  y: n device floats.  For testing. */
+spade_status spade_selftest_exp2_poly(const float* x, float* y, int n, spade_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -122,8 +122,12 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __r
 }
 
 // ------------------------------------------------------------ work list --
-// Items (head, query block) ranked by cost = number of key blocks walked,
-// descending (longest first), by a counting sort in one CTA.
+// Items (head, query block) in head-major order; inside a head, ranked by
+// cost = number of key blocks walked, descending (longest first), by a
+// counting sort -- one CTA per head.  Consecutive items then share a head, so
+// the K/V blocks that persistent attention CTAs work on at any time stay
+// L2-resident, and long lists start before short ones.  CTA 0 also resets the
+// ticket the attention kernel hands the list out with.
 struct WorklistArgs {
   int heads;
   int ntb;
@@ -134,15 +138,7 @@ struct WorklistArgs {
   int cnt_off[SPADE_MAX_HEADS];
 };
 
-__device__ __forceinline__ void decode_item(const WorklistArgs& a, int g, int& h, int& qb) {
-  int lo = 0, hi = a.heads - 1;
-  while (lo < hi) {                               // last head with item_start <= g
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.item_start[mid] <= g) lo = mid; else hi = mid - 1;
-  }
-  h = lo;
-  qb = g - a.item_start[lo];
-}
+constexpr int kWlThreads = 512;
 
 __device__ __forceinline__ int item_cost(const WorklistArgs& a, const int* cnt, int h, int qb) {
   const int nb = a.nb[h];
@@ -150,22 +146,25 @@ __device__ __forceinline__ int item_cost(const WorklistArgs& a, const int* cnt, 
   return cnt[a.cnt_off[h] + qb] + a.ntb;
 }
 
-__global__ void __launch_bounds__(1024) worklist_kernel(const __grid_constant__ WorklistArgs a,
-                                                        const int* __restrict__ cnt, int* __restrict__ work) {
+__global__ void __launch_bounds__(kWlThreads) worklist_kernel(const __grid_constant__ WorklistArgs a,
+                                                              const int* __restrict__ cnt,
+                                                              int* __restrict__ work, int* __restrict__ ticket) {
   __shared__ int hist[SPADE_WORKLIST_MAX_COST];
-  __shared__ int warp_tot[32];
+  __shared__ int warp_tot[kWlThreads / 32];
   const int tid = threadIdx.x;
-  for (int i = tid; i < SPADE_WORKLIST_MAX_COST; i += blockDim.x) hist[i] = 0;
+  const int h = blockIdx.x;
+  if (h == 0 && tid == 0) *ticket = 0;
+  const int base = a.item_start[h];
+  const int n = a.item_start[h + 1] - base;
+  for (int i = tid; i < SPADE_WORKLIST_MAX_COST; i += kWlThreads) hist[i] = 0;
   __syncthreads();
-  for (int g = tid; g < a.n_items; g += blockDim.x) {
-    int h, qb;
-    decode_item(a, g, h, qb);
+  for (int qb = tid; qb < n; qb += kWlThreads) {
     const int c = min(item_cost(a, cnt, h, qb), SPADE_WORKLIST_MAX_COST - 1);
     atomicAdd(&hist[SPADE_WORKLIST_MAX_COST - 1 - c], 1);
   }
   __syncthreads();
-  // exclusive scan over bins: each thread owns 4 consecutive bins
-  constexpr int PER = SPADE_WORKLIST_MAX_COST / 1024;
+  // exclusive scan over bins: each thread owns PER consecutive bins
+  constexpr int PER = SPADE_WORKLIST_MAX_COST / kWlThreads;
   int local[PER];
   int s = 0;
 #pragma unroll
@@ -180,25 +179,23 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const __grid_constant__ 
   if (lane == 31) warp_tot[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_tot[lane];
+    int w = lane < kWlThreads / 32 ? warp_tot[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int t = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += t;
     }
-    warp_tot[lane] = w;
+    if (lane < kWlThreads / 32) warp_tot[lane] = w;
   }
   __syncthreads();
-  int base = inc - s + (warp > 0 ? warp_tot[warp - 1] : 0);
+  int off = inc - s + (warp > 0 ? warp_tot[warp - 1] : 0);
 #pragma unroll
-  for (int e = 0; e < PER; ++e) { hist[tid * PER + e] = base; base += local[e]; }
+  for (int e = 0; e < PER; ++e) { hist[tid * PER + e] = off; off += local[e]; }
   __syncthreads();
-  for (int g = tid; g < a.n_items; g += blockDim.x) {
-    int h, qb;
-    decode_item(a, g, h, qb);
+  for (int qb = tid; qb < n; qb += kWlThreads) {
     const int c = min(item_cost(a, cnt, h, qb), SPADE_WORKLIST_MAX_COST - 1);
     const int pos = atomicAdd(&hist[SPADE_WORKLIST_MAX_COST - 1 - c], 1);
-    work[pos] = (h << 16) | qb;
+    work[base + pos] = (h << 16) | qb;
   }
 }
 
@@ -239,7 +236,7 @@ cudaError_t launch_worklist(const AttnArgs& a, cudaStream_t s) {
   }
   w.item_start[a.heads] = acc;
   w.n_items = acc;
-  worklist_kernel<<<1, 1024, 0, s>>>(w, a.cnt, a.work);
+  worklist_kernel<<<a.heads, kWlThreads, 0, s>>>(w, a.cnt, a.work, a.ticket);
   return cudaGetLastError();
 }
 

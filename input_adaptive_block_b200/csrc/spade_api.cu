@@ -84,6 +84,7 @@ struct GroupLayout {
   size_t cnt[SPADE_MAX_SCHEMES], idx[SPADE_MAX_SCHEMES];
   std::vector<int> pos;                             // position of head h in its scheme group
   size_t work;
+  size_t ticket;
   int n_items;
   size_t total;
 };
@@ -133,6 +134,8 @@ spade_status plan_group(const spade_geom* schemes, int n_schemes, const spade_he
   }
   L.work = off;
   off = align256(off + (size_t)L.n_items * sizeof(int));
+  L.ticket = off;
+  off = align256(off + sizeof(int));
   L.total = off;
   return SPADE_OK;
 }
@@ -256,7 +259,7 @@ size_t spade_attn_workspace_bytes(spade_geom g, int heads, int d, int text_token
   if (heads < 1 || text_tokens < 0 || g.bt <= 0 || g.bh <= 0 || g.bw <= 0 || g.T <= 0 || g.H <= 0 || g.W <= 0)
     return 0;
   const Geo gg = make_geo(g);
-  return align256((size_t)heads * (gg.nb + text_blocks(text_tokens)) * sizeof(int));
+  return align256((size_t)heads * (gg.nb + text_blocks(text_tokens)) * sizeof(int)) + 256;   // + ticket
 }
 
 spade_status spade_block_sparse_attn(const void* q, const void* k, const void* v, void* out, const int* cnt,
@@ -290,6 +293,7 @@ spade_status spade_block_sparse_attn(const void* q, const void* k, const void* v
   a.cnt = cnt; a.idx = idx;
   a.work = static_cast<int*>(workspace);
   a.n_items = heads * (nb + text_blocks(text_tokens));
+  a.ticket = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + need - 256);
   return run_attention(a, as_cuda(stream));
 }
 
@@ -376,6 +380,7 @@ spade_status spade_grouped_attn(const void* q, const void* k, const void* v, voi
   a.cnt = reinterpret_cast<const int*>(ws);
   a.idx = reinterpret_cast<const int*>(ws);
   a.work = reinterpret_cast<int*>(ws + L.work);
+  a.ticket = reinterpret_cast<int*>(ws + L.ticket);
   a.n_items = L.n_items;
   return run_attention(a, s);
 }
@@ -398,6 +403,13 @@ spade_status spade_selftest_bounded_wait(int64_t timeout_ns, spade_stream_t stre
   if (!sp) return fail(SPADE_ERR_CUDA, "device status word unavailable");
   cudaError_t e = launch_bounded_wait_selftest(sp, timeout_ns, as_cuda(stream));
   return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "bounded-wait self test");
+}
+
+spade_status spade_selftest_exp2_poly(const float* x, float* y, int n, spade_stream_t stream) {
+  if (!x || !y || n < 0) return fail(SPADE_ERR_INVALID, "null pointer or negative n");
+  if (n == 0) return SPADE_OK;
+  cudaError_t e = launch_exp2_poly_selftest(x, y, n, as_cuda(stream));
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "exp2 polynomial self test");
 }
 
 }  // extern "C"

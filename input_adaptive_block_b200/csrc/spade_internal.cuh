@@ -13,6 +13,7 @@
 #define SPADE_SELECT_MAX_HEADS 1024
 #define SPADE_ESTIMATE_MAX_NB 2048
 #define SPADE_WORKLIST_MAX_COST 4096
+#define SPADE_TC_MAX_LIST 1280   // tensor-core path: key blocks per item (nb + text blocks)
 
 namespace spade {
 
@@ -65,6 +66,7 @@ struct AttnArgs {
   const int* cnt;      // base of the kept counts
   const int* idx;      // base of the kept ids
   int* work;           // [n_items] work list (built on device)
+  int* ticket;         // one int next to the work list: dynamic work hand-out
   int n_items;
   spade_dtype dt;
   int* status;         // device status word
@@ -89,6 +91,7 @@ cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 bool attn_tc_supported(const AttnArgs& a);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s, const char** why);
 cudaError_t launch_bounded_wait_selftest(int* status, long long timeout_ns, cudaStream_t s);
+cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int n, cudaStream_t s);
 
 int num_sms();                               // SM count of the current device
 long long device_wait_timeout_ns();          // limit for every bounded device wait
