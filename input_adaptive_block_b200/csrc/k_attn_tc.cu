@@ -59,12 +59,13 @@ struct Cfg {
   static constexpr int OFF_PLIST = OFF_KV + NS * TILE;            // producer's copy of the key list
   static constexpr int OFF_SEXT = OFF_PLIST + 4 * kMaxList;       // softmax warps: extent code per block
   static constexpr int OFF_DEC = OFF_SEXT + 4 * kMaxList;         // slot -> (t, y, x) per scheme
-  static constexpr int OFF_BAR = OFF_DEC + 4 * 128 * SPADE_MAX_SCHEMES;
+  static constexpr int OFF_RED = OFF_DEC + 4 * 128 * SPADE_MAX_SCHEMES;  // row max / sum exchange
+  static constexpr int OFF_BAR = OFF_RED + 4 * (2 * 2 * 128 + 2 * 128);
   static constexpr int SMEM = OFF_BAR + 512 + 1024;               // barriers + alignment slack
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
   static constexpr uint32_t COL_P0 = 256 + D, COL_P1 = 256 + D + 64;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;   // producer, MMA, 8 softmax warps
 };
 
 struct __align__(64) TcParams {
@@ -117,18 +118,19 @@ struct Waiter {
   long long timeout_ns;
 };
 
+// Waiting threads sleep in try_wait (hardware suspend, woken when the phase
+// completes) rather than spin: the producer and MMA warps share schedulers
+// with two of the softmax warps, and a spinning waiter steals their issue slots.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Waiter& w) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*w.abort) return false;
-      if ((long long)(ptx::globaltimer() - t0) > w.timeout_ns) {
-        *w.abort = 1;
-        atomicExch(w.status, (int)SPADE_ERR_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (ptx::mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (*w.abort) return false;
+    if ((long long)(ptx::globaltimer() - t0) > w.timeout_ns) {
+      *w.abort = 1;
+      atomicExch(w.status, (int)SPADE_ERR_TIMEOUT);
+      return false;
     }
   }
 }
@@ -167,17 +169,30 @@ __device__ __forceinline__ int key_block(const TcParams& p, const Item& I, int k
   return I.nb + (k - I.ncnt);
 }
 
-template <int D>
-__device__ __forceinline__ void load_tile(const TcParams& p, const CUtensorMap* vid, const CUtensorMap* txt,
-                                          const Item& I, int blk, uint8_t* dst, uint64_t* bar) {
+// Packed tile coordinates of key block `blk`, decoded once per work item so
+// the producer's per-tile path has no integer division: video blocks keep
+// (bk, bj, bi) in bits 0-11 / 12-21 / 22-30, text blocks set bit 31 and keep
+// their index in the low bits.
+__device__ __forceinline__ uint32_t pack_coord(const TcParams& p, const Item& I, int blk) {
   if (blk < I.nb) {
     const Geo& g = p.geo[I.scheme];
     const int bk = blk % g.nbw, bj = (blk / g.nbw) % g.nbh, bi = blk / (g.nbw * g.nbh);
+    return (uint32_t)bk | ((uint32_t)bj << 12) | ((uint32_t)bi << 22);
+  }
+  return 0x80000000u | (uint32_t)(blk - I.nb);
+}
+
+template <int D>
+__device__ __forceinline__ void load_tile(const TcParams& p, const CUtensorMap* vid, const CUtensorMap* txt,
+                                          const Item& I, uint32_t pc, uint8_t* dst, uint64_t* bar) {
+  if (!(pc & 0x80000000u)) {
+    const Geo& g = p.geo[I.scheme];
+    const int bk = (int)(pc & 0xfffu), bj = (int)((pc >> 12) & 0x3ffu), bi = (int)(pc >> 22);
 #pragma unroll
     for (int a = 0; a < D / 64; ++a)
       ptx::tma_load_5d_elect(dst + a * kAtomBytes, vid, bar, 64 * a, I.h, bk * g.bw, bj * g.bh, bi * g.bt);
   } else {
-    const int tb = blk - I.nb;
+    const int tb = (int)(pc & 0x7fffffffu);
 #pragma unroll
     for (int a = 0; a < D / 64; ++a) ptx::tma_load_3d_elect(dst + a * kAtomBytes, txt, bar, 64 * a, I.h, tb * 128);
   }
@@ -250,9 +265,11 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sKV = smem + C::OFF_KV;
-  int* plist = reinterpret_cast<int*>(smem + C::OFF_PLIST);
+  int* plist = reinterpret_cast<int*>(smem + C::OFF_PLIST);   // packed tile coordinates
   uint32_t* sext = reinterpret_cast<uint32_t*>(smem + C::OFF_SEXT);
   uint32_t* sdec = reinterpret_cast<uint32_t*>(smem + C::OFF_DEC);
+  float* pmax = reinterpret_cast<float*>(smem + C::OFF_RED);   // [2 parity][2 halves][128 rows]
+  float* psum = pmax + 2 * 2 * 128;                             // [2 halves][128 rows]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + C::NS;
@@ -265,7 +282,10 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
   uint64_t* mma_fin = q_full + 11;
   uint64_t* item_full = q_full + 12;
   uint64_t* item_empty = item_full + kItemRing;
-  int* item_ring = reinterpret_cast<int*>(item_empty + kItemRing);
+  uint64_t* xbar = item_empty + kItemRing;      // [quad][block parity]: partner row-max exchange
+  uint64_t* ebar = xbar + 8;                    // [quad]: partner row-sum exchange (epilogue)
+  uint64_t* stage_bar = ebar + 4;               // softmax warps: key-list extents staged
+  int* item_ring = reinterpret_cast<int*>(stage_bar + 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_ring + kItemRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -284,15 +304,18 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
       ptx::mbar_init(&q_full[b], 1);
       ptx::mbar_init(&q_empty[b], 1);
       ptx::mbar_init(&s_full[b], 1);
-      ptx::mbar_init(&p_full[b], 128);
+      ptx::mbar_init(&p_full[b], 256);
       ptx::mbar_init(&pv_done[b], 1);
     }
-    ptx::mbar_init(o_free, 128);
+    ptx::mbar_init(o_free, 256);
     ptx::mbar_init(mma_fin, 1);
     for (int r = 0; r < kItemRing; ++r) {
       ptx::mbar_init(&item_full[r], 1);
-      ptx::mbar_init(&item_empty[r], 1 + 128);   // the MMA thread and every softmax thread
+      ptx::mbar_init(&item_empty[r], 1 + 256);   // the MMA warp and every softmax thread
     }
+    for (int r = 0; r < 8; ++r) ptx::mbar_init(&xbar[r], 64);
+    for (int r = 0; r < 4; ++r) ptx::mbar_init(&ebar[r], 64);
+    ptx::mbar_init(stage_bar, 256);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -341,20 +364,20 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
       __syncwarp();
       if (it < 0) break;
       const Item I = get_item(p, it);
-      for (int j = lane; j < I.n; j += 32) plist[j] = key_block(p, I, j);
+      for (int j = lane; j < I.n; j += 32) plist[j] = (int)pack_coord(p, I, key_block(p, I, j));
       __syncwarp();
       const int qs = li % C::NQ;
       ok = __all_sync(0xffffffffu, wait_bar(&q_empty[qs], ((li / C::NQ) & 1) ^ 1, W));
       if (!ok) break;
       ptx::mbar_arrive_expect_tx_elect(&q_full[qs], C::TILE);
-      load_tile<D>(p, &p.tm_q[I.scheme], &p.tm_qt, I, I.qb, sQ + qs * C::TILE, &q_full[qs]);
+      load_tile<D>(p, &p.tm_q[I.scheme], &p.tm_qt, I, pack_coord(p, I, I.qb), sQ + qs * C::TILE, &q_full[qs]);
       qlast[qs] = (li / C::NQ) & 1;
-      auto push = [&](const CUtensorMap* vid, const CUtensorMap* txt, int blk) -> bool {
+      auto push = [&](const CUtensorMap* vid, const CUtensorMap* txt, int pcw) -> bool {
         const int st = kvpos % C::NS;
         const uint32_t par = (kvpos / C::NS) & 1;
         if (!__all_sync(0xffffffffu, wait_bar(&kv_empty[st], par ^ 1, W))) return false;
         ptx::mbar_arrive_expect_tx_elect(&kv_full[st], C::TILE);
-        load_tile<D>(p, vid, txt, I, blk, sKV + st * C::TILE, &kv_full[st]);
+        load_tile<D>(p, vid, txt, I, (uint32_t)pcw, sKV + st * C::TILE, &kv_full[st]);
         last_par[st] = par;
         used |= 1u << st;
         ++kvpos;
@@ -453,10 +476,17 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
     drain_bar(mma_fin, 0, 100000000LL);
   } else {
     // ---------------------------------------- softmax / correction / epilogue --
+    // Eight warps, two per TMEM lane quadrant: warp half hf owns score columns
+    // [64 hf, 64 hf + 64) of the quadrant's 32 rows (and the same half of O).
+    // The two partners (same quadrant, same scheduler) exchange their partial
+    // row maxima through shared memory, so both use the same running max; row
+    // sums stay per half and are combined in the epilogue.
+    constexpr int OH = D / 2;                          // O columns per half
+    const int hf = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;                  // TMEM lane = query slot
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    const int stid = threadIdx.x - 64;                 // 0..127 within the softmax warps
+    const int stid = threadIdx.x - 64;                 // 0..255 within the softmax warps
     const float sl2 = p.scale_log2;
     const float2 sl2x2 = make_float2(sl2, sl2);
     uint32_t g = 0;
@@ -469,44 +499,52 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
       ptx::mbar_arrive(&item_empty[slot]);
       if (it < 0) break;
       const Item I = get_item(p, it);
-      for (int j = stid; j < I.n; j += 128) sext[j] = extent_code(p, I, key_block(p, I, j));
-      ptx::named_bar_sync(1, 128);
+      for (int j = stid; j < I.n; j += 256) sext[j] = extent_code(p, I, key_block(p, I, j));
+      ptx::mbar_arrive(stage_bar);
+      ok = wait_bar(stage_bar, li & 1, W);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       const uint32_t* dec = sdec + 128 * I.scheme;
-      float m_use = 0.f, l = 0.f;
+      float m_use = 0.f, l = 0.f;                      // l: this half's share of the row sum
       for (int j = 0; j < I.n; ++j) {
         const uint32_t gj = g + j, b = gj & 1;
         ok = wait_bar(&s_full[b], (gj >> 1) & 1, W);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         ptx::tc_fence_after();
-        uint32_t sr[128];
-        ptx::tmem_ld128(tmem + lane_base + (b ? C::COL_S1 : C::COL_S0), sr);
+        uint32_t sr[64];
+        ptx::tmem_ld64(tmem + lane_base + (b ? C::COL_S1 : C::COL_S0) + 64 * hf, sr);
         const uint32_t code = sext[j];
         const bool full = (code & kFullBlock) != 0;
-        uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
         if (!full) {
+          uint32_t mw[4];
           key_mask(code, dec, lane, mw);
+          const uint32_t w0 = hf ? mw[2] : mw[0], w1 = hf ? mw[3] : mw[1];
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (!((mw[c >> 5] >> (c & 31)) & 1u)) sr[c] = 0xff800000u;   // -inf
+          for (int c = 0; c < 64; ++c)
+            if (!((((c < 32) ? w0 : w1) >> (c & 31)) & 1u)) sr[c] = 0xff800000u;   // -inf
         }
-        // row max: eight independent chains of 3-input max
+        // partial row max (eight 3-input chains), then the partner's half
         float mk[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) mk[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]));
 #pragma unroll
-        for (int c = 16; c < 128; c += 16) {
+        for (int c = 16; c < 64; c += 16) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             mk[k] = max3f(mk[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + k + 8]));
         }
-        const float mx =
-            max3f(max3f(mk[0], mk[1], mk[2]), max3f(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7])) * sl2;
+        const float pm = max3f(max3f(mk[0], mk[1], mk[2]), max3f(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
+        float* px = pmax + (b * 2) * 128;
+        px[hf * 128 + row] = pm;
+        ptx::mbar_arrive(&xbar[quad * 2 + b]);
+        ok = wait_bar(&xbar[quad * 2 + b], (gj >> 1) & 1, W);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        const float mx = fmaxf(pm, px[(1 - hf) * 128 + row]) * sl2;
         if (j == 0) {
           m_use = mx;
         } else {
           const bool need = mx > m_use + 8.0f;
           if (__any_sync(0xffffffffu, need)) {
-            // rescale O by 2^(m_use - mx) once PV(j-1) has landed
+            // rescale this half of O by 2^(m_use - mx) once PV(j-1) has landed
             const uint32_t gp = gj - 1;
             ok = wait_bar(&pv_done[gp & 1], (gp >> 1) & 1, W);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -514,12 +552,13 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
             const float alpha = need ? ptx::ex2(m_use - mx) : 1.0f;
             if (need) { l *= alpha; m_use = mx; }
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = 0; c0 < OH; c0 += 32) {
               uint32_t ob[32];
-              ptx::tmem_ld32(tmem + lane_base + C::COL_O + c0, ob);
+              const uint32_t ta = tmem + lane_base + C::COL_O + OH * hf + c0;
+              ptx::tmem_ld32(ta, ob);
 #pragma unroll
               for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(__uint_as_float(ob[c]) * alpha);
-              ptx::tmem_st32(tmem + lane_base + C::COL_O + c0, ob);
+              ptx::tmem_st32(ta, ob);
             }
           }
         }
@@ -527,12 +566,12 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
         // straight-line so the SFU ops pipeline back to back (masked columns
         // are -inf and give an exact 0)
         const float2 nm2 = make_float2(-m_use, -m_use);
-        float2 pe[64];
+        float2 pe[32];
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < 32; ++c)
           pe[c] = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2, nm2);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < 32; ++c) {
           pe[c].x = ptx::ex2(pe[c].x);
           pe[c].y = ptx::ex2(pe[c].y);
         }
@@ -540,30 +579,34 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] = pe[k];
 #pragma unroll
-        for (int c = 8; c < 64; ++c) acc[c & 7] = __fadd2_rn(acc[c & 7], pe[c]);
+        for (int c = 8; c < 32; ++c) acc[c & 7] = __fadd2_rn(acc[c & 7], pe[c]);
         const float2 a = __fadd2_rn(__fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3])),
                                     __fadd2_rn(__fadd2_rn(acc[4], acc[5]), __fadd2_rn(acc[6], acc[7])));
         l += a.x + a.y;
-        uint32_t pk[64];
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) pk[c] = ptx::pack_bf16x2(pe[c].x, pe[c].y);
+        for (int c = 0; c < 32; ++c) pk[c] = ptx::pack_bf16x2(pe[c].x, pe[c].y);
         if (j >= 2) {                                  // P buffer b was read by PV(j-2)
           const uint32_t gp = gj - 2;
           ok = wait_bar(&pv_done[b], (gp >> 1) & 1, W);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         }
-        const uint32_t tP = tmem + lane_base + (b ? C::COL_P1 : C::COL_P0);
-        ptx::tmem_st64(tP, pk);
+        ptx::tmem_st32(tmem + lane_base + (b ? C::COL_P1 : C::COL_P0) + 32 * hf, pk);
         ptx::tc_fence_before();
         ptx::mbar_arrive(&p_full[b]);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16, each thread stores its own query row straight
-      // to token order (padded slots of edge blocks are skipped)
+      // epilogue: O / l -> bf16, each thread stores its half of its query row
+      // straight to token order (padded slots of edge blocks are skipped)
       const uint32_t gl = g + I.n - 1;
       ok = wait_bar(&pv_done[gl & 1], (gl >> 1) & 1, W);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       ptx::tc_fence_after();
+      psum[hf * 128 + row] = l;
+      ptx::mbar_arrive(&ebar[quad]);
+      ok = wait_bar(&ebar[quad], li & 1, W);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      const float inv = 1.0f / (l + psum[(1 - hf) * 128 + row]);
       long long tok = -1;
       if (I.qb < I.nb) {
         const Geo& gg = p.geo[I.scheme];
@@ -576,12 +619,12 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
         const int t = (I.qb - I.nb) * 128 + row;
         if (t < p.text_tokens) tok = (long long)p.N + t;
       }
-      const float inv = 1.0f / l;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + ((tok < 0 ? 0 : tok) * p.heads + I.h) * (long long)(D * 2));
+      uint4* dst = reinterpret_cast<uint4*>(p.out + ((tok < 0 ? 0 : tok) * p.heads + I.h) * (long long)(D * 2) +
+                                            OH * 2 * hf);
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < OH; c0 += 32) {
         uint32_t ov[32];
-        ptx::tmem_ld32(tmem + lane_base + C::COL_O + c0, ov);
+        ptx::tmem_ld32(tmem + lane_base + C::COL_O + OH * hf + c0, ov);
         if (tok >= 0) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
@@ -658,8 +701,10 @@ cudaError_t launch_d(const TcParams& tp, int grid, cudaStream_t s) {
 
 bool attn_tc_supported(const AttnArgs& a) {
   if (a.dt != SPADE_BF16 || (a.d != 64 && a.d != 128)) return false;
-  for (int s = 0; s < a.n_schemes; ++s)
+  for (int s = 0; s < a.n_schemes; ++s) {
     if (a.geo[s].bs != 128) return false;
+    if (a.geo[s].nbw >= 4096 || a.geo[s].nbh >= 1024 || a.geo[s].nbt >= 512) return false;   // packed coords
+  }
   const int ntb = text_blocks(a.text_tokens);
   for (int h = 0; h < a.heads; ++h)
     if (a.head[h].nb + ntb > kMaxList) return false;
