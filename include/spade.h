@@ -133,6 +133,30 @@ spade_status spade_block_sparse_attn(const void* q, const void* k, const void* v
                                      int heads, int d, int text_tokens, spade_dtype dt,
                                      void* workspace, size_t ws_bytes, spade_stream_t stream);
 
+/* ---- step 5 without a caller workspace ------------------------------------
+ * Not from the SPADE pages (they have no counterpart): the same computation
+ * and arguments as spade_block_sparse_attn, minus the workspace, for callers
+ * that cannot allocate device memory themselves -- for example code running
+ * where another component owns every allocation, or a runtime that forbids
+ * allocation on the call path.  The per-call scratch (the work list and its
+ * hand-out counter) lives instead in one fixed device array inside the
+ * library: 65536 work items (256 KiB), held on every device that uses it
+ * until the library is unloaded.
+ *  - heads * (nb + ceil(text_tokens/128)) must be <= 65536; larger calls
+ *    return SPADE_ERR_UNSUPPORTED and enqueue nothing.
+ *  - The library allocates nothing here (no cudaMalloc/cudaFree).  The first
+ *    call on each device looks up the array's device address (with that
+ *    device current) and caches it; make that first call before any stream
+ *    capture.
+ *  - Every call shares the one array, and each call rewrites it in full
+ *    (the counter is reset on the device at the start of each call).  Calls
+ *    whose work overlaps on the GPU -- on different streams, or from
+ *    different threads -- race on it; order them (one stream, or events). */
+spade_status spade_block_sparse_attn_noalloc(const void* q, const void* k, const void* v, void* out,
+                                             const int* cnt, const int* idx, spade_geom g,
+                                             int heads, int d, int text_tokens, spade_dtype dt,
+                                             spade_stream_t stream);
+
 /* ---- steps 1-5 for heads of mixed schemes, one grouped attention launch ---
  * Methodology 3, "Head Grouping"; abstract, "kernel grouping".  Runs the
  * summarizer, estimator and index search per scheme for the non-dense heads,

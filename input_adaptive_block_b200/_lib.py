@@ -34,6 +34,8 @@ SIGNATURES = {
     "spade_block_sparse_attn": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                         SpadeGeom, c_int, c_int, c_int, c_int, c_void_p, c_size_t,
                                         c_void_p]),
+    "spade_block_sparse_attn_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                SpadeGeom, c_int, c_int, c_int, c_int, c_void_p]),
     "spade_grouped_workspace_bytes": (c_size_t, [POINTER(SpadeGeom), c_int, POINTER(SpadeHeadScheme),
                                                  c_int, c_int, c_int]),
     "spade_grouped_attn": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SpadeGeom), c_int,

@@ -16,7 +16,7 @@ from ._lib import SpadeGeom, SpadeHeadScheme, check
 
 __all__ = [
     "geom", "dtype_code", "tile3d", "summarize", "estimate", "select", "attn_workspace_bytes",
-    "block_sparse_attn", "grouped_workspace_bytes", "grouped_attn", "grouped_head_lists",
+    "block_sparse_attn", "block_sparse_attn_noalloc", "grouped_workspace_bytes", "grouped_attn", "grouped_head_lists",
     "last_device_status", "selftest_bounded_wait", "num_blocks",
 ]
 
@@ -117,6 +117,24 @@ def block_sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cnt: Op
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), cp, ip, gg, heads, d, text_tokens,
         dtype_code(q.dtype), _dev(workspace, "workspace"), workspace.numel(), _stream(stream)),
         "spade_block_sparse_attn")
+    return out
+
+
+def block_sparse_attn_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cnt: Optional[torch.Tensor],
+                              idx: Optional[torch.Tensor], g, text_tokens: int = 0,
+                              out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """spade_block_sparse_attn without a workspace argument: the library keeps
+    the scratch in a fixed device array of its own (see include/spade.h for
+    the size limit and the rule that overlapping calls must be ordered)."""
+    gg = geom(g)
+    heads, d = q.shape[1], q.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    cp = _dev(cnt, "cnt") if cnt is not None else None
+    ip = _dev(idx, "idx") if idx is not None else None
+    check(_lib.load().spade_block_sparse_attn_noalloc(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), cp, ip, gg, heads, d, text_tokens,
+        dtype_code(q.dtype), _stream(stream)), "spade_block_sparse_attn_noalloc")
     return out
 
 

@@ -13,6 +13,12 @@
 // Latched device status (SPADE_OK / SPADE_ERR_TIMEOUT), one per device.
 __device__ int g_spade_status;
 
+// Fixed scratch for spade_block_sparse_attn_noalloc: the cost-ranked work list
+// (up to SPADE_NOALLOC_MAX_ITEMS entries) followed by the work-hand-out ticket.
+// Lives for as long as the library is loaded, on every device that uses it.
+#define SPADE_NOALLOC_MAX_ITEMS 65536
+static __device__ __align__(256) int g_noalloc_scratch[SPADE_NOALLOC_MAX_ITEMS + 64];
+
 namespace spade {
 
 namespace {
@@ -158,6 +164,28 @@ spade_status run_attention(AttnArgs& a, cudaStream_t s) {
   return SPADE_OK;
 }
 
+// Device address of g_noalloc_scratch on the current device.  The name is only
+// a host-side stand-in in host code, so the address is looked up once per
+// device (with that device current) and cached.
+int* noalloc_scratch(spade_status* st) {
+  static int* ptrs[kMaxDevices] = {nullptr};
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) {
+    *st = fail(SPADE_ERR_CUDA, "no current CUDA device");
+    return nullptr;
+  }
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) {
+      *st = cuda_fail(e, "fixed scratch address");
+      return nullptr;
+    }
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
 }  // namespace
 
 int num_sms() {
@@ -294,6 +322,45 @@ spade_status spade_block_sparse_attn(const void* q, const void* k, const void* v
   a.work = static_cast<int*>(workspace);
   a.n_items = heads * (nb + text_blocks(text_tokens));
   a.ticket = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + need - 256);
+  return run_attention(a, as_cuda(stream));
+}
+
+spade_status spade_block_sparse_attn_noalloc(const void* q, const void* k, const void* v, void* out,
+                                             const int* cnt, const int* idx, spade_geom g, int heads, int d,
+                                             int text_tokens, spade_dtype dt, spade_stream_t stream) {
+  spade_status st = check_geom(g);
+  if (st != SPADE_OK) return st;
+  if ((st = check_d_dt(d, dt)) != SPADE_OK) return st;
+  if (!q || !k || !v || !out) return fail(SPADE_ERR_INVALID, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  if ((cnt == nullptr) != (idx == nullptr)) return fail(SPADE_ERR_INVALID, "cnt and idx must both be set or both NULL");
+  if (heads < 1 || heads > SPADE_MAX_HEADS) return fail(SPADE_ERR_UNSUPPORTED, "heads=%d (1..128)", heads);
+  if (text_tokens < 0) return fail(SPADE_ERR_INVALID, "negative text_tokens");
+  const int nb = make_geo(g).nb;
+  const long long n_items = (long long)heads * (nb + text_blocks(text_tokens));
+  if (n_items > SPADE_NOALLOC_MAX_ITEMS)
+    return fail(SPADE_ERR_UNSUPPORTED, "heads * (blocks + text blocks) = %lld exceeds the fixed scratch of %d work items",
+                n_items, SPADE_NOALLOC_MAX_ITEMS);
+  int* scratch = noalloc_scratch(&st);
+  if (!scratch) return st;
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out;
+  a.n_schemes = 1;
+  a.geo[0] = make_geo(g);
+  a.heads = heads; a.d = d; a.text_tokens = text_tokens; a.N = g.T * g.H * g.W; a.dt = dt;
+  for (int h = 0; h < heads; ++h) {
+    a.head[h].scheme = 0;
+    a.head[h].nb = nb;
+    a.head[h].dense = cnt == nullptr;
+    a.head[h].cnt_off = h * nb;
+    a.head[h].idx_off = (long long)h * nb * nb;
+  }
+  a.cnt = cnt; a.idx = idx;
+  a.work = scratch;                                   // written in full by the work-list kernel
+  a.ticket = scratch + SPADE_NOALLOC_MAX_ITEMS;       // reset to 0 by the work-list kernel
+  a.n_items = (int)n_items;
   return run_attention(a, as_cuda(stream));
 }
 
