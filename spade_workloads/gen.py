@@ -106,26 +106,29 @@ def torch_dtype(wl: Workload) -> torch.dtype:
 
 
 def make_qkv(wl: Workload, device="cpu", heads: Optional[int] = None,
-             out_dtype: Optional[torch.dtype] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """Q, K, V as [N + text, heads, d] tensors in the workload dtype."""
-    h_count = wl.heads if heads is None else heads
+             out_dtype: Optional[torch.dtype] = None,
+             head_list: Optional[list] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Q, K, V as [N + text, heads, d] tensors in the workload dtype.  With
+    head_list, only those heads are generated (slot i holds head head_list[i]);
+    each head's values do not depend on which other heads are generated."""
+    hl = list(head_list) if head_list is not None else list(range(wl.heads if heads is None else heads))
     dt = torch_dtype(wl) if out_dtype is None else out_dtype
     n_tot = wl.n_total
     outs = []
     for tensor in (TENSOR_Q, TENSOR_K, TENSOR_V):
-        out = torch.empty(n_tot, h_count, wl.d, dtype=dt, device=device)
-        for h in range(h_count):
+        out = torch.empty(n_tot, len(hl), wl.d, dtype=dt, device=device)
+        for slot, h in enumerate(hl):
             noise = counter_normal(stream_key(wl.config_id, tensor, h), wl.N * wl.d, device)
             noise = noise.view(wl.N, wl.d)
             if tensor == TENSOR_V:
                 vals = noise
             else:
                 vals = smooth_field(wl, tensor, h, device) + 0.5 * noise
-            out[: wl.N, h, :] = vals.to(dt)
+            out[: wl.N, slot, :] = vals.to(dt)
             if wl.text_tokens:
                 tk = stream_key(wl.config_id, tensor + _TEXT_OFFSET, h)
                 txt = counter_normal(tk, wl.text_tokens * wl.d, device).view(wl.text_tokens, wl.d)
-                out[wl.N:, h, :] = txt.to(dt)
+                out[wl.N:, slot, :] = txt.to(dt)
             del noise, vals
         outs.append(out)
     return outs[0], outs[1], outs[2]
