@@ -11,17 +11,25 @@
 //    map {d, head, x, y, t} with box {64, 1, bw, bh, bt} lands one block of one
 //    head in shared memory as 128 rows x 128 B (slot order t, y, x), 128-byte
 //    swizzled -- the layout the MMA reads.  Out-of-grid slots are zero-filled
-//    by the TMA unit; the output goes back through the same map, and the TMA
-//    store clips padded rows.  No tiled copy of Q/K/V is ever written.
-//  * tcgen05.mma (kind::f16, bf16 in, fp32 accumulate), issued by one thread:
-//    S = Q K^T (128x128, both operands in shared memory) into one of two TMEM
-//    buffers; O += P V with P (bf16) read from TMEM and V from shared memory.
-//  * Warp specialisation: warp 0 loads (TMA) and hands out work, warp 1 issues
-//    MMAs, warps 2-5 own one TMEM lane (query row) each: masked online
-//    softmax (exp2 domain, lazy rescaling of O only when the running max grows
-//    by more than 2^8), P back to TMEM, epilogue (O / l -> bf16 -> swizzled
-//    smem -> TMA store).  A quarter of the exponentials of full blocks run on
-//    the FMA pipe (polynomial, below) so the SFU does not bound the softmax.
+//    by the TMA unit.  No tiled copy of Q/K/V is ever written.
+//  * tcgen05.mma (kind::f16, bf16 in, fp32 accumulate), issued by one thread.
+//    TMEM (512 columns): S0 | S1 (scores of key blocks j even / odd, fp32) |
+//    O (fp32) | P0 | P1 (bf16 probabilities).  S(j+2) is computed as soon as
+//    the softmax has read S(j) into registers (and is issued ahead of the
+//    other group's P V), so a score tile is normally waiting when the softmax
+//    reaches it; P V runs behind, reading P from TMEM.
+//  * Warp specialisation: warp 0 hands out work and issues TMA loads (one K/V
+//    ring), warp 1 issues the Q K^T MMAs and warp 2 the P V MMAs (so neither
+//    stream's waits hold back the other's issue), warps 3-6 and 7-10 are two
+//    softmax warpgroups taking the even and the odd kept blocks of
+//    the query tile: each thread owns one query row (TMEM lane) with all 128
+//    key columns.  The two groups accumulate into one O, so they share a
+//    per-row reference maximum through shared memory: block j reads the
+//    reference left by block j-1 (a short handshake), raises it only when its
+//    own row maximum is more than 2^8 above (then rescales O once the P V
+//    issued before it has landed), and every block's P is taken relative to
+//    that reference.  Row sums stay per group and are combined in the epilogue
+//    (O / l -> bf16 -> token order; each group writes half of the columns).
 //  * Persistent CTAs take (head, query block) items from a work list ordered
 //    head-major (longest first within a head) through an atomic ticket: the
 //    K/V blocks in use at any time belong to one or two heads and stay in L2,
@@ -31,7 +39,6 @@
 //    draining its own TMA loads and MMAs before freeing TMEM.
 #include <cudaTypedefs.h>
 
-#include <cstdlib>
 
 #include "ptx.cuh"
 #include "spade_internal.cuh"
@@ -45,27 +52,28 @@ constexpr int kItemRing = 4;                 // work items in flight between the
 constexpr uint32_t kFullBlock = 1u << 31;    // extent code: every slot valid
 constexpr uint32_t kTextBlock = 1u << 30;    // extent code: text block (low bits = valid count)
 
-template <int D, int NQ_, int NS_>
+// POLY_: when 1, every fourth column pair's exponential runs on the FMA pipe
+template <int D, int NS_, int POLY_>
 struct Cfg {
-  static constexpr int ATOMS = D / 64;
   static constexpr int TILE = 128 * D * 2;
   // K/V ring stages (TMA latency under load is ~1-1.5 us, so the ring holds
-  // several (query tile, key block) pairs of look-ahead); shared memory use
-  // keeps one CTA per SM, which owns all 512 TMEM columns
+  // several key blocks of look-ahead); shared memory use keeps one CTA per
+  // SM, which owns all 512 TMEM columns
   static constexpr int NS = NS_;
-  static constexpr int NQ = NQ_;                                  // Q buffers
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = NQ * TILE;
+  static constexpr int OFF_KV = TILE;
   static constexpr int OFF_PLIST = OFF_KV + NS * TILE;            // producer's copy of the key list
-  static constexpr int OFF_SEXT = OFF_PLIST + 4 * kMaxList;       // softmax warps: extent code per block
+  static constexpr int OFF_SEXT = OFF_PLIST + 4 * kMaxList;       // softmax: extent code per block
   static constexpr int OFF_DEC = OFF_SEXT + 4 * kMaxList;         // slot -> (t, y, x) per scheme
-  static constexpr int OFF_RED = OFF_DEC + 4 * 128 * SPADE_MAX_SCHEMES;  // row max / sum exchange
-  static constexpr int OFF_BAR = OFF_RED + 4 * (2 * 2 * 128 + 2 * 128);
+  static constexpr int OFF_MREF = OFF_DEC + 4 * 128 * SPADE_MAX_SCHEMES;   // per-row reference max
+  static constexpr int OFF_LX = OFF_MREF + 4 * 128;               // [2 groups][128 rows] row sums
+  static constexpr int OFF_BAR = OFF_LX + 4 * 2 * 128;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;               // barriers + alignment slack
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O = 256;
-  static constexpr uint32_t COL_P0 = 256 + D, COL_P1 = 256 + D + 64;
+  static constexpr uint32_t COL_S = 0;                            // S(j) at 128 (j % 2)
+  static constexpr uint32_t COL_O = 256;
+  static constexpr uint32_t COL_P = 256 + D;                      // P(j) at COL_P + 64 (j % 2)
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 320;   // producer, MMA, 8 softmax warps
+  static constexpr int THREADS = 352;   // producer, two MMA issuers, two softmax warpgroups
 };
 
 struct __align__(64) TcParams {
@@ -258,9 +266,9 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-template <int D, int NQ, int NS>
-__global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
-  using C = Cfg<D, NQ, NS>;
+template <int D, int NS, int POLY>
+__global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
+  using C = Cfg<D, NS, POLY>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
@@ -268,24 +276,26 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
   int* plist = reinterpret_cast<int*>(smem + C::OFF_PLIST);   // packed tile coordinates
   uint32_t* sext = reinterpret_cast<uint32_t*>(smem + C::OFF_SEXT);
   uint32_t* sdec = reinterpret_cast<uint32_t*>(smem + C::OFF_DEC);
-  float* pmax = reinterpret_cast<float*>(smem + C::OFF_RED);   // [2 parity][2 halves][128 rows]
-  float* psum = pmax + 2 * 2 * 128;                             // [2 halves][128 rows]
+  float* mref = reinterpret_cast<float*>(smem + C::OFF_MREF);  // [128 rows] reference max (log2 domain)
+  float* lx = reinterpret_cast<float*>(smem + C::OFF_LX);      // [2 groups][128 rows] final row sums
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars;
-  uint64_t* kv_empty = bars + C::NS;
-  uint64_t* q_full = bars + 2 * C::NS;
-  uint64_t* q_empty = q_full + 2;
-  uint64_t* s_full = q_full + 4;
-  uint64_t* p_full = q_full + 6;
-  uint64_t* pv_done = q_full + 8;
-  uint64_t* o_free = q_full + 10;
-  uint64_t* mma_fin = q_full + 11;
-  uint64_t* item_full = q_full + 12;
+  uint64_t* kv_empty = bars + NS;
+  uint64_t* q_full = bars + 2 * NS;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* s_full = q_full + 2;      // [2] S(j) in TMEM (MMA commit)
+  uint64_t* s_free = q_full + 4;      // [2] S(j) read by its group (128 threads)
+  uint64_t* p_full = q_full + 6;      // [2] P(j) in TMEM (128 threads)
+  uint64_t* pv_done = q_full + 8;     // [2] P V(j) complete (MMA commit)
+  uint64_t* md = q_full + 10;         // [2] reference max of block j final (128 threads of its group)
+  uint64_t* o_full = q_full + 12;     // last P V of the item complete
+  uint64_t* o_free = q_full + 13;     // epilogue has read O (256 threads)
+  uint64_t* lx_bar = q_full + 14;     // both groups' final row sums published (256 threads)
+  uint64_t* stage_bar = q_full + 15;  // extent codes of the item staged (256 threads)
+  uint64_t* mma_fin = q_full + 16;    // [2] per MMA warp: all its MMAs complete
+  uint64_t* item_full = q_full + 18;
   uint64_t* item_empty = item_full + kItemRing;
-  uint64_t* xbar = item_empty + kItemRing;      // [quad][block parity]: partner row-max exchange
-  uint64_t* ebar = xbar + 8;                    // [quad]: partner row-sum exchange (epilogue)
-  uint64_t* stage_bar = ebar + 4;               // softmax warps: key-list extents staged
-  int* item_ring = reinterpret_cast<int*>(stage_bar + 1);
+  int* item_ring = reinterpret_cast<int*>(item_empty + kItemRing);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_ring + kItemRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -296,26 +306,29 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
     sdec[e] = (uint32_t)(c / (g.bw * g.bh)) | ((uint32_t)((c / g.bw) % g.bh) << 8) | ((uint32_t)(c % g.bw) << 16);
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NS; ++s) {
+    for (int s = 0; s < NS; ++s) {
       ptx::mbar_init(&kv_full[s], 1);
       ptx::mbar_init(&kv_empty[s], 1);
     }
+    ptx::mbar_init(q_full, 1);
+    ptx::mbar_init(q_empty, 1);
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(&q_full[b], 1);
-      ptx::mbar_init(&q_empty[b], 1);
       ptx::mbar_init(&s_full[b], 1);
-      ptx::mbar_init(&p_full[b], 256);
+      ptx::mbar_init(&s_free[b], 128);
+      ptx::mbar_init(&p_full[b], 128);
       ptx::mbar_init(&pv_done[b], 1);
+      ptx::mbar_init(&md[b], 128);
     }
+    ptx::mbar_init(o_full, 1);
     ptx::mbar_init(o_free, 256);
-    ptx::mbar_init(mma_fin, 1);
+    ptx::mbar_init(lx_bar, 256);
+    ptx::mbar_init(stage_bar, 256);
+    ptx::mbar_init(&mma_fin[0], 1);
+    ptx::mbar_init(&mma_fin[1], 1);
     for (int r = 0; r < kItemRing; ++r) {
       ptx::mbar_init(&item_full[r], 1);
-      ptx::mbar_init(&item_empty[r], 1 + 256);   // the MMA warp and every softmax thread
+      ptx::mbar_init(&item_empty[r], 2 + 256);   // both MMA warps and every softmax thread
     }
-    for (int r = 0; r < 8; ++r) ptx::mbar_init(&xbar[r], 64);
-    for (int r = 0; r < 4; ++r) ptx::mbar_init(&ebar[r], 64);
-    ptx::mbar_init(stage_bar, 256);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -342,10 +355,11 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
     // item's key list in shared memory; one elected lane takes the ticket,
     // publishes the item (or -1 at the end) to the other roles, and issues
     // each expect-tx / TMA load (elect.sync-predicated, no divergent branch).
+    // Ring order = MMA consumption order: K0, K1, K2, then K_{j+3}, V_j.
     uint32_t kvpos = 0;
-    uint32_t last_par[C::NS];
+    uint32_t last_par[NS];
     uint32_t used = 0;
-    int qlast[2] = {-1, -1};
+    int qlast = -1;
     bool ok = true;
     for (int li = 0;; ++li) {
       int it = 0;
@@ -366,15 +380,14 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
       const Item I = get_item(p, it);
       for (int j = lane; j < I.n; j += 32) plist[j] = (int)pack_coord(p, I, key_block(p, I, j));
       __syncwarp();
-      const int qs = li % C::NQ;
-      ok = __all_sync(0xffffffffu, wait_bar(&q_empty[qs], ((li / C::NQ) & 1) ^ 1, W));
+      ok = __all_sync(0xffffffffu, wait_bar(q_empty, (li & 1) ^ 1, W));
       if (!ok) break;
-      ptx::mbar_arrive_expect_tx_elect(&q_full[qs], C::TILE);
-      load_tile<D>(p, &p.tm_q[I.scheme], &p.tm_qt, I, pack_coord(p, I, I.qb), sQ + qs * C::TILE, &q_full[qs]);
-      qlast[qs] = (li / C::NQ) & 1;
+      ptx::mbar_arrive_expect_tx_elect(q_full, C::TILE);
+      load_tile<D>(p, &p.tm_q[I.scheme], &p.tm_qt, I, pack_coord(p, I, I.qb), sQ, q_full);
+      qlast = li & 1;
       auto push = [&](const CUtensorMap* vid, const CUtensorMap* txt, int pcw) -> bool {
-        const int st = kvpos % C::NS;
-        const uint32_t par = (kvpos / C::NS) & 1;
+        const int st = kvpos % NS;
+        const uint32_t par = (kvpos / NS) & 1;
         if (!__all_sync(0xffffffffu, wait_bar(&kv_empty[st], par ^ 1, W))) return false;
         ptx::mbar_arrive_expect_tx_elect(&kv_full[st], C::TILE);
         load_tile<D>(p, vid, txt, I, (uint32_t)pcw, sKV + st * C::TILE, &kv_full[st]);
@@ -383,30 +396,39 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
         ++kvpos;
         return true;
       };
-      // ring order = MMA consumption order: K0, K1, then K_{j+2}, V_j
-      for (int j = 0; ok && j < 2 && j < I.n; ++j) ok = push(&p.tm_k[I.scheme], &p.tm_kt, plist[j]);
+      for (int j = 0; ok && j < 3 && j < I.n; ++j) ok = push(&p.tm_k[I.scheme], &p.tm_kt, plist[j]);
       for (int j = 0; ok && j < I.n; ++j) {
-        if (j + 2 < I.n) ok = push(&p.tm_k[I.scheme], &p.tm_kt, plist[j + 2]);
+        if (j + 3 < I.n) ok = push(&p.tm_k[I.scheme], &p.tm_kt, plist[j + 3]);
         if (ok) ok = push(&p.tm_v[I.scheme], &p.tm_vt, plist[j]);
       }
       __syncwarp();
       if (!ok) break;
     }
     if (lane == 0 && !ok) {   // wind down: let every load this warp issued land before the CTA exits
-      for (int st = 0; st < C::NS; ++st)
+      for (int st = 0; st < NS; ++st)
         if (used & (1u << st)) drain_bar(&kv_full[st], last_par[st], 100000000LL);
-      for (int b = 0; b < C::NQ; ++b)
-        if (qlast[b] >= 0) drain_bar(&q_full[b], qlast[b], 100000000LL);
+      if (qlast >= 0) drain_bar(q_full, qlast, 100000000LL);
     }
-  } else if (warp == 1) {
-    // -------------------------------------------------------- MMA issuer --
-    // The whole warp runs this loop in uniform control flow (waits, item
-    // bookkeeping, descriptors); one elected lane issues each tcgen05.mma /
-    // commit.  Issuing from a lane-divergent region costs a register-to-
-    // uniform conversion per MMA, which is slower than the MMA itself.
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------- MMA issuers --
+    // Warp 1 issues the score MMAs S(k) = Q K_k^T, warp 2 the P V(j) MMAs.
+    // The two streams touch disjoint TMEM (S buffers vs P buffers and O) and
+    // each commit tracks only its own warp's MMAs, so each warp blocks only on
+    // its own events: S(k) waits for its K tile and for the group that owns
+    // S buffer k % 2 to have read S(k-2); P V(j) waits for P(j) and V_j.  One
+    // warp waiting never holds back the other's issue, which keeps the
+    // (shallow) tensor instruction queue fed.  Each warp runs in uniform
+    // control flow; one elected lane issues each tcgen05.mma / commit.
+    //
+    // Ring positions inside an item with n blocks (base B): K_k at B + k for
+    // k < 3, at B + m + 2 (k - 3) otherwise; V_j at B + m + min(j + 1, n - 3) + j,
+    // where m = min(n, 3) -- the producer's order K0, K1, K2, then K_{j+3}, V_j.
+    const bool is_s = warp == 1;
     constexpr uint32_t idesc_qk = make_idesc(128, 128, false);
     constexpr uint32_t idesc_pv = make_idesc(128, D, true);
-    uint32_t kvpos = 0, g = 0;
+    uint32_t base = 0;         // ring position of the item's first tile
+    uint32_t su[2] = {0, 0};   // S writes per buffer so far (S warp)
+    uint32_t pu[2] = {0, 0};   // P V reads per buffer so far (P V warp)
     bool ok = true;
     for (int li = 0; ok; ++li) {
       const int slot = li % kItemRing;
@@ -416,80 +438,77 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&item_empty[slot]);
       if (it < 0) break;
-      const Item I = get_item(p, it);
-      const int qs = li % C::NQ;
-      ok = wait_bar(&q_full[qs], (li / C::NQ) & 1, W);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      ptx::tc_fence_after();
-      const uint64_t qdesc = kmajor_desc(ptx::smem_u32(sQ + qs * C::TILE));
-      // S(j) -> S buffer j%2, P(j) -> P buffer j%2.  Once softmax(j) has
-      // published P(j) (and so released S buffer j%2), S(j+2) is issued ahead
-      // of PV(j), so the next-but-one score tile is ready as early as possible.
-      auto issue_s = [&](int jj) -> bool {
-        const int st = kvpos % C::NS;
-        if (!__all_sync(0xffffffffu, wait_bar(&kv_full[st], (kvpos / C::NS) & 1, W))) return false;
+      const int n = get_item(p, it).n;
+      const int m = n < 3 ? n : 3;
+      const int nk3 = n > 3 ? n - 3 : 0;
+      if (is_s) {
+        ok = wait_bar(q_full, li & 1, W);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         ptx::tc_fence_after();
-        const uint32_t b = (g + jj) & 1;
-        const uint64_t kdesc = kmajor_desc(ptx::smem_u32(sKV + st * C::TILE));
-        const uint32_t ts = tmem + (b ? C::COL_S1 : C::COL_S0);
+        const uint64_t qdesc = kmajor_desc(ptx::smem_u32(sQ));
+        for (int k = 0; ok && k < n; ++k) {
+          const int b = k & 1;
+          const uint32_t pos = base + (uint32_t)(k < 3 ? k : m + 2 * (k - 3));
+          const int st = (int)(pos % NS);
+          bool w = wait_bar(&kv_full[st], (pos / NS) & 1, W);
+          if (su[b] > 0) w = w && wait_bar(&s_free[b], (su[b] - 1) & 1, W);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint64_t kdesc = kmajor_desc(ptx::smem_u32(sKV + st * C::TILE));
+          const uint32_t ts = tmem + C::COL_S + 128 * b;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * kAtomBytes + (kk & 3) * 32) >> 4);
-          ptx::mma_ss_elect(ts, qdesc + off, kdesc + off, idesc_qk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * kAtomBytes + (kk & 3) * 32) >> 4);
+            ptx::mma_ss_elect(ts, qdesc + off, kdesc + off, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          ptx::tc_commit_elect(&s_full[b]);
+          ptx::tc_commit_elect(&kv_empty[st]);
+          ++su[b];
+          if (k == n - 1) ptx::tc_commit_elect(q_empty);
         }
-        ptx::tc_commit_elect(&s_full[b]);
-        ptx::tc_commit_elect(&kv_empty[st]);
-        ++kvpos;
-        if (jj == I.n - 1) ptx::tc_commit_elect(&q_empty[qs]);
-        return true;
-      };
-      auto issue_pv = [&](int jj) -> bool {
-        const uint32_t b = (g + jj) & 1;
-        const int st = kvpos % C::NS;
-        bool w = wait_bar(&kv_full[st], (kvpos / C::NS) & 1, W);
-        if (jj == 0) w = w && wait_bar(o_free, (li & 1) ^ 1, W);
-        if (!__all_sync(0xffffffffu, w)) return false;
-        ptx::tc_fence_after();
-        const uint64_t vdesc = mnmajor_desc(ptx::smem_u32(sKV + st * C::TILE));
-        const uint32_t tp = tmem + (b ? C::COL_P1 : C::COL_P0);
-        const uint32_t acc0 = jj > 0 ? 1u : 0u;
+      } else {
+        for (int j = 0; ok && j < n; ++j) {
+          const int b = j & 1;
+          const uint32_t pos = base + (uint32_t)(m + (j + 1 < nk3 ? j + 1 : nk3) + j);
+          const int st = (int)(pos % NS);
+          bool w = wait_bar(&p_full[b], pu[b] & 1, W);
+          w = w && wait_bar(&kv_full[st], (pos / NS) & 1, W);
+          if (j == 0) w = w && wait_bar(o_free, (li & 1) ^ 1, W);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint64_t vdesc = mnmajor_desc(ptx::smem_u32(sKV + st * C::TILE));
+          const uint32_t tp = tmem + C::COL_P + 64 * b;
+          const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          ptx::mma_ts_elect(tmem + C::COL_O, tp + kk * 8, vdesc + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
-                            kk > 0 ? 1u : acc0);
-        ptx::tc_commit_elect(&pv_done[b]);
-        ptx::tc_commit_elect(&kv_empty[st]);
-        ++kvpos;
-        return true;
-      };
-      for (int j = 0; ok && j < 2 && j < I.n; ++j) ok = issue_s(j);
-      for (int j = 0; ok && j < I.n; ++j) {
-        const uint32_t gj = g + j;
-        ok = __all_sync(0xffffffffu, wait_bar(&p_full[gj & 1], (gj >> 1) & 1, W));
-        if (ok && j + 2 < I.n) ok = issue_s(j + 2);
-        if (ok) ok = issue_pv(j);
+          for (int kk = 0; kk < 8; ++kk)
+            ptx::mma_ts_elect(tmem + C::COL_O, tp + kk * 8, vdesc + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
+                              kk > 0 ? 1u : acc0);
+          ptx::tc_commit_elect(&pv_done[b]);
+          ptx::tc_commit_elect(&kv_empty[st]);
+          ++pu[b];
+          if (j == n - 1) ptx::tc_commit_elect(o_full);
+        }
       }
-      g += I.n;
+      base += 2u * (uint32_t)n;
     }
     // every MMA this warp issued completes before TMEM is released
-    ptx::tc_commit_elect(mma_fin);
-    drain_bar(mma_fin, 0, 100000000LL);
+    ptx::tc_commit_elect(&mma_fin[is_s ? 0 : 1]);
+    drain_bar(&mma_fin[is_s ? 0 : 1], 0, 100000000LL);
   } else {
-    // ---------------------------------------- softmax / correction / epilogue --
-    // Eight warps, two per TMEM lane quadrant: warp half hf owns score columns
-    // [64 hf, 64 hf + 64) of the quadrant's 32 rows (and the same half of O).
-    // The two partners (same quadrant, same scheduler) exchange their partial
-    // row maxima through shared memory, so both use the same running max; row
-    // sums stay per half and are combined in the epilogue.
-    constexpr int OH = D / 2;                          // O columns per half
-    const int hf = (warp - 2) >> 2;
+    // ------------------------------------------------ softmax / epilogue --
+    // Group w (warps 3-6: w = 0, warps 7-10: w = 1) takes the item's blocks
+    // j with j % 2 == w.  Thread = one query row (TMEM lane), all 128 columns.
+    const int w = (warp - 3) >> 2;
     const int quad = warp & 3;
-    const int row = quad * 32 + lane;                  // TMEM lane = query slot
+    const int row = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    const int stid = threadIdx.x - 64;                 // 0..255 within the softmax warps
+    const int gtid = threadIdx.x - 96;                 // 0..255 over both groups
+    const uint32_t tS = tmem + lane_base + C::COL_S + 128 * w;
+    const uint32_t tP = tmem + lane_base + C::COL_P + 64 * w;
+    const uint32_t tO = tmem + lane_base + C::COL_O;
     const float sl2 = p.scale_log2;
     const float2 sl2x2 = make_float2(sl2, sl2);
-    uint32_t g = 0;
+    uint32_t nb_done[2] = {0, 0};                      // blocks of each group before this item
     bool ok = true;
     for (int li = 0; ok; ++li) {
       const int slot = li % kItemRing;
@@ -499,148 +518,178 @@ __global__ void __launch_bounds__(Cfg<D, NQ, NS>::THREADS, 1) attn_tc_kernel(con
       ptx::mbar_arrive(&item_empty[slot]);
       if (it < 0) break;
       const Item I = get_item(p, it);
-      for (int j = stid; j < I.n; j += 256) sext[j] = extent_code(p, I, key_block(p, I, j));
+      const int n = I.n;
+      // both groups finished the previous item (its row sums were exchanged
+      // after their last block), so the codes can be overwritten
+      for (int j = gtid; j < n; j += 256) sext[j] = extent_code(p, I, key_block(p, I, j));
       ptx::mbar_arrive(stage_bar);
       ok = wait_bar(stage_bar, li & 1, W);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       const uint32_t* dec = sdec + 128 * I.scheme;
-      float m_use = 0.f, l = 0.f;                      // l: this half's share of the row sum
-      for (int j = 0; j < I.n; ++j) {
-        const uint32_t gj = g + j, b = gj & 1;
-        ok = wait_bar(&s_full[b], (gj >> 1) & 1, W);
+      float l = 0.f;          // this group's share of the row sum, relative to m_seen
+      float m_seen = 0.f;     // reference max at this group's last block
+      for (int j = w; j < n; j += 2) {
+        const uint32_t kself = nb_done[w] + (uint32_t)(j >> 1);        // this group's block counter
+        ok = wait_bar(&s_full[w], kself & 1, W);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         ptx::tc_fence_after();
-        uint32_t sr[64];
-        ptx::tmem_ld64(tmem + lane_base + (b ? C::COL_S1 : C::COL_S0) + 64 * hf, sr);
+        uint32_t sr[128];
+        ptx::tmem_ld128(tS, sr);
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&s_free[w]);                  // S buffer may take S(j+2)
         const uint32_t code = sext[j];
-        const bool full = (code & kFullBlock) != 0;
-        if (!full) {
+        if (!(code & kFullBlock)) {
           uint32_t mw[4];
           key_mask(code, dec, lane, mw);
-          const uint32_t w0 = hf ? mw[2] : mw[0], w1 = hf ? mw[3] : mw[1];
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (!((((c < 32) ? w0 : w1) >> (c & 31)) & 1u)) sr[c] = 0xff800000u;   // -inf
+          for (int c = 0; c < 128; ++c)
+            if (!((mw[c >> 5] >> (c & 31)) & 1u)) sr[c] = 0xff800000u;   // -inf
         }
-        // partial row max (eight 3-input chains), then the partner's half
         float mk[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) mk[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[k + 8]));
 #pragma unroll
-        for (int c = 16; c < 64; c += 16) {
+        for (int c = 16; c < 128; c += 16) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             mk[k] = max3f(mk[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + k + 8]));
         }
-        const float pm = max3f(max3f(mk[0], mk[1], mk[2]), max3f(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
-        float* px = pmax + (b * 2) * 128;
-        px[hf * 128 + row] = pm;
-        ptx::mbar_arrive(&xbar[quad * 2 + b]);
-        ok = wait_bar(&xbar[quad * 2 + b], (gj >> 1) & 1, W);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        const float mx = fmaxf(pm, px[(1 - hf) * 128 + row]) * sl2;
-        if (j == 0) {
-          m_use = mx;
-        } else {
-          const bool need = mx > m_use + 8.0f;
-          if (__any_sync(0xffffffffu, need)) {
-            // rescale this half of O by 2^(m_use - mx) once PV(j-1) has landed
-            const uint32_t gp = gj - 1;
-            ok = wait_bar(&pv_done[gp & 1], (gp >> 1) & 1, W);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            ptx::tc_fence_after();
-            const float alpha = need ? ptx::ex2(m_use - mx) : 1.0f;
-            if (need) { l *= alpha; m_use = mx; }
-#pragma unroll 1
-            for (int c0 = 0; c0 < OH; c0 += 32) {
-              uint32_t ob[32];
-              const uint32_t ta = tmem + lane_base + C::COL_O + OH * hf + c0;
-              ptx::tmem_ld32(ta, ob);
-#pragma unroll
-              for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(__uint_as_float(ob[c]) * alpha);
-              ptx::tmem_st32(ta, ob);
-            }
+        const float mx = max3f(max3f(mk[0], mk[1], mk[2]), max3f(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7])) * sl2;
+        // reference max: block 0 sets it; block j > 0 reads what block j-1
+        // left and raises it only when its own max is more than 2^8 above
+        float m_use = mx, alpha = 1.0f;
+        bool raise = false;
+        if (j > 0) {
+          const uint32_t kother = nb_done[w ^ 1] + (uint32_t)((j - 1) >> 1);   // block j-1's index in its group
+          ok = wait_bar(&md[w ^ 1], kother & 1, W);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          const float mprev = mref[row];
+          if (mx > mprev + 8.0f) {
+            raise = true;
+            alpha = ptx::ex2(mprev - mx);
+          } else {
+            m_use = mprev;
           }
         }
-        // p = 2^(s*scale*log2e - m): one FFMA2 per column pair, then the SFU,
-        // straight-line so the SFU ops pipeline back to back (masked columns
-        // are -inf and give an exact 0)
-        const float2 nm2 = make_float2(-m_use, -m_use);
-        float2 pe[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          pe[c] = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), sl2x2, nm2);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          pe[c].x = ptx::ex2(pe[c].x);
-          pe[c].y = ptx::ex2(pe[c].y);
-        }
-        float2 acc[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = pe[k];
-#pragma unroll
-        for (int c = 8; c < 32; ++c) acc[c & 7] = __fadd2_rn(acc[c & 7], pe[c]);
-        const float2 a = __fadd2_rn(__fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3])),
-                                    __fadd2_rn(__fadd2_rn(acc[4], acc[5]), __fadd2_rn(acc[6], acc[7])));
-        l += a.x + a.y;
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = ptx::pack_bf16x2(pe[c].x, pe[c].y);
-        if (j >= 2) {                                  // P buffer b was read by PV(j-2)
-          const uint32_t gp = gj - 2;
-          ok = wait_bar(&pv_done[b], (gp >> 1) & 1, W);
+        if (j == 0 || raise) mref[row] = m_use;
+        ptx::mbar_arrive(&md[w]);
+        if (l != 0.f && m_seen != m_use) l *= ptx::ex2(m_seen - m_use);
+        m_seen = m_use;
+        // P buffer w was last read by this group's previous block's P V
+        if (kself > 0) {
+          ok = wait_bar(&pv_done[w], (kself - 1) & 1, W);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         }
-        ptx::tmem_st32(tmem + lane_base + (b ? C::COL_P1 : C::COL_P0) + 32 * hf, pk);
+        // p = 2^(s*scale*log2e - m) in four 32-column chunks: FFMA2, exp2
+        // (SFU; with POLY, every fourth pair on the FMA pipe), row-sum FADD2,
+        // bf16 pack, TMEM store; masked columns are -inf and give 0
+        {
+          const float2 nm2 = make_float2(-m_use, -m_use);
+          float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                            make_float2(0.f, 0.f)};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float2 pe[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              pe[c] = __ffma2_rn(
+                  make_float2(__uint_as_float(sr[32 * q + 2 * c]), __uint_as_float(sr[32 * q + 2 * c + 1])), sl2x2, nm2);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              if (POLY && (c & 3) == 3) {
+                pe[c] = exp2_poly2(pe[c]);
+              } else {
+                pe[c].x = ptx::ex2(pe[c].x);
+                pe[c].y = ptx::ex2(pe[c].y);
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 16; ++c) acc4[c & 3] = __fadd2_rn(acc4[c & 3], pe[c]);
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk[c] = ptx::pack_bf16x2(pe[c].x, pe[c].y);
+            ptx::tmem_st16_nowait(tP + 16 * q, pk);
+          }
+          const float2 a = __fadd2_rn(__fadd2_rn(acc4[0], acc4[1]), __fadd2_rn(acc4[2], acc4[3]));
+          l += a.x + a.y;
+        }
+        ptx::tmem_wait_st();
+        if (__any_sync(0xffffffffu, raise)) {
+          // O holds blocks < j relative to the old reference: rescale it once
+          // P V(j-1) has landed (P V(j) waits for this group's P below)
+          const uint32_t kother = nb_done[w ^ 1] + (uint32_t)((j - 1) >> 1);
+          ok = wait_bar(&pv_done[w ^ 1], kother & 1, W);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          ptx::tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ob[32];
+            ptx::tmem_ld32(tO + c0, ob);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(__uint_as_float(ob[c]) * alpha);
+            ptx::tmem_st32(tO + c0, ob);
+          }
+        }
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&p_full[b]);
+        ptx::mbar_arrive(&p_full[w]);
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16, each thread stores its half of its query row
-      // straight to token order (padded slots of edge blocks are skipped)
-      const uint32_t gl = g + I.n - 1;
-      ok = wait_bar(&pv_done[gl & 1], (gl >> 1) & 1, W);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      ptx::tc_fence_after();
-      psum[hf * 128 + row] = l;
-      ptx::mbar_arrive(&ebar[quad]);
-      ok = wait_bar(&ebar[quad], li & 1, W);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      const float inv = 1.0f / (l + psum[(1 - hf) * 128 + row]);
+      // ---- epilogue: combine the groups' row sums, O / l -> bf16 -> token order
+      {
+        const int jl = n - 1;                          // last block: its reference max is final
+        if ((jl & 1) != w) {
+          const uint32_t kl = nb_done[w ^ 1] + (uint32_t)(jl >> 1);
+          ok = wait_bar(&md[w ^ 1], kl & 1, W);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        }
+        const float mfin = mref[row];
+        if (l != 0.f && m_seen != mfin) l *= ptx::ex2(m_seen - mfin);
+        lx[w * 128 + row] = l;
+        ptx::mbar_arrive(lx_bar);
+        ok = wait_bar(lx_bar, li & 1, W);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        ok = wait_bar(o_full, li & 1, W);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        ptx::tc_fence_after();
+      }
+      nb_done[0] += (uint32_t)((n + 1) >> 1);
+      nb_done[1] += (uint32_t)(n >> 1);
+      const float inv = 1.0f / (lx[row] + lx[128 + row]);
+      const Item E = get_item(p, it);   // re-read: nothing of the item stays live across the block loop
       long long tok = -1;
-      if (I.qb < I.nb) {
-        const Geo& gg = p.geo[I.scheme];
+      if (E.qb < E.nb) {
+        const Geo& gg = p.geo[E.scheme];
         int t0, y0, x0, et, eh, ew;
-        block_box(gg, I.qb, t0, y0, x0, et, eh, ew);
-        const uint32_t e = dec[row];
+        block_box(gg, E.qb, t0, y0, x0, et, eh, ew);
+        const uint32_t e = sdec[128 * E.scheme + row];
         const int tl = (int)(e & 0xffu), yl = (int)((e >> 8) & 0xffu), xl = (int)(e >> 16);
         if (tl < et && yl < eh && xl < ew) tok = ((long long)(t0 + tl) * gg.H + (y0 + yl)) * gg.W + (x0 + xl);
       } else {
-        const int t = (I.qb - I.nb) * 128 + row;
+        const int t = (E.qb - E.nb) * 128 + row;
         if (t < p.text_tokens) tok = (long long)p.N + t;
       }
-      uint4* dst = reinterpret_cast<uint4*>(p.out + ((tok < 0 ? 0 : tok) * p.heads + I.h) * (long long)(D * 2) +
-                                            OH * 2 * hf);
-#pragma unroll
+      constexpr int OH = D / 2;                        // this group's output columns
+      uint4* dst = reinterpret_cast<uint4*>(p.out + ((tok < 0 ? 0 : tok) * p.heads + E.h) * (long long)(D * 2) +
+                                            OH * 2 * w);
+#pragma unroll 1
       for (int c0 = 0; c0 < OH; c0 += 32) {
         uint32_t ov[32];
-        ptx::tmem_ld32(tmem + lane_base + C::COL_O + OH * hf + c0, ov);
+        ptx::tmem_ld32(tO + OH * w + c0, ov);
         if (tok >= 0) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             const int c = q4 * 8;
-            uint4 w;
-            w.x = ptx::pack_bf16x2(__uint_as_float(ov[c + 0]) * inv, __uint_as_float(ov[c + 1]) * inv);
-            w.y = ptx::pack_bf16x2(__uint_as_float(ov[c + 2]) * inv, __uint_as_float(ov[c + 3]) * inv);
-            w.z = ptx::pack_bf16x2(__uint_as_float(ov[c + 4]) * inv, __uint_as_float(ov[c + 5]) * inv);
-            w.w = ptx::pack_bf16x2(__uint_as_float(ov[c + 6]) * inv, __uint_as_float(ov[c + 7]) * inv);
-            dst[c0 / 8 + q4] = w;
+            uint4 v4;
+            v4.x = ptx::pack_bf16x2(__uint_as_float(ov[c + 0]) * inv, __uint_as_float(ov[c + 1]) * inv);
+            v4.y = ptx::pack_bf16x2(__uint_as_float(ov[c + 2]) * inv, __uint_as_float(ov[c + 3]) * inv);
+            v4.z = ptx::pack_bf16x2(__uint_as_float(ov[c + 4]) * inv, __uint_as_float(ov[c + 5]) * inv);
+            v4.w = ptx::pack_bf16x2(__uint_as_float(ov[c + 6]) * inv, __uint_as_float(ov[c + 7]) * inv);
+            dst[c0 / 8 + q4] = v4;
           }
         }
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(o_free);
-      g += I.n;
     }
   }
 
@@ -686,14 +735,14 @@ bool map_text(CUtensorMap* m, const void* base, int text, int heads, int d) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int NQ, int NS>
+template <int D, int NS, int POLY>
 cudaError_t launch_d(const TcParams& tp, int grid, cudaStream_t s) {
-  using C = Cfg<D, NQ, NS>;
+  using C = Cfg<D, NS, POLY>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
   cudaError_t e =
-      cudaFuncSetAttribute(attn_tc_kernel<D, NQ, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+      cudaFuncSetAttribute(attn_tc_kernel<D, NS, POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<D, NQ, NS><<<grid, C::THREADS, C::SMEM, s>>>(tp);
+  attn_tc_kernel<D, NS, POLY><<<grid, C::THREADS, C::SMEM, s>>>(tp);
   return cudaGetLastError();
 }
 
@@ -754,10 +803,8 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s, const char** why) 
   tp.timeout_ns = device_wait_timeout_ns();
   const int grid = a.n_items < num_sms() ? a.n_items : num_sms();
   if (grid <= 0) return cudaSuccess;
-  if (a.d == 64) return launch_d<64, 2, 8>(tp, grid, s);
-  const char* v = getenv("SPADE_TC_VARIANT");   // ring-depth experiment (temporary)
-  if (v && v[0] == '1') return launch_d<128, 2, 4>(tp, grid, s);
-  return launch_d<128, 1, 5>(tp, grid, s);
+  if (a.d == 64) return launch_d<64, 8, 0>(tp, grid, s);
+  return launch_d<128, 5, 0>(tp, grid, s);
 }
 
 // ------------------------------------------------- bounded-wait self test --

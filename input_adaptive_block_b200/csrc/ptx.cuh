@@ -288,6 +288,16 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t* r) {
       SPADE_W8(0), SPADE_W8(8), SPADE_W8(16), SPADE_W8(24), SPADE_W8(32), SPADE_W8(40), SPADE_W8(48), SPADE_W8(56)
       : "memory");
 }
+// r[0..15] -> 16 consecutive TMEM columns of this thread's lane, no wait
+// (pair with tmem_wait_st before the columns are handed to another agent).
+__device__ __forceinline__ void tmem_st16_nowait(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      SPADE_W8(0), SPADE_W8(8)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 #undef SPADE_R8
 #undef SPADE_W8
 
