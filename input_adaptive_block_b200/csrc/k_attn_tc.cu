@@ -20,8 +20,8 @@
 //    reaches it; P V runs behind, reading P from TMEM.
 //  * Warp specialisation: warp 0 hands out work and issues TMA loads (one K/V
 //    ring), warp 1 issues the Q K^T MMAs and warp 2 the P V MMAs (so neither
-//    stream's waits hold back the other's issue), warps 3-6 and 7-10 are two
-//    softmax warpgroups taking the even and the odd kept blocks of
+//    stream's waits hold back the other's issue), warps 4-7 and 8-11 are two
+//    softmax warpgroups (with most of the register file: setmaxnreg) taking the even and the odd kept blocks of
 //    the query tile: each thread owns one query row (TMEM lane) with all 128
 //    key columns.  The two groups accumulate into one O, so they share a
 //    per-row reference maximum through shared memory: block j reads the
@@ -73,7 +73,13 @@ struct Cfg {
   static constexpr uint32_t COL_O = 256;
   static constexpr uint32_t COL_P = 256 + D;                      // P(j) at COL_P + 64 (j % 2)
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 352;   // producer, two MMA issuers, two softmax warpgroups
+  // warpgroup 0: producer, two MMA issuers, one idle warp; warpgroups 1-2:
+  // softmax.  Registers per thread after the split (setmaxnreg): the split
+  // must fit in the launch-time pool of THREADS x (registers per thread).
+  static constexpr int THREADS = 384;
+  static constexpr int REG_CTRL = 56;
+  static constexpr int REG_SOFTMAX = 208;
+  static constexpr int REG_POOL_NEEDED = 128 * REG_CTRL + 256 * REG_SOFTMAX;
 };
 
 struct __align__(64) TcParams {
@@ -348,8 +354,12 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.timeout_ns};
-
-  if (warp == 0) {
+  if (warp < 4) {
+  // ------------------------------------------------ warpgroup 0: control --
+  ptx::setmaxnreg_dec<C::REG_CTRL>();
+  if (warp == 3) {
+    // idle: its registers went to the softmax warpgroups
+  } else if (warp == 0) {
     // ------------------------------------------- scheduler + TMA producer --
     // The whole warp runs this loop in uniform control flow and stages each
     // item's key list in shared memory; one elected lane takes the ticket,
@@ -494,15 +504,17 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
     // every MMA this warp issued completes before TMEM is released
     ptx::tc_commit_elect(&mma_fin[is_s ? 0 : 1]);
     drain_bar(&mma_fin[is_s ? 0 : 1], 0, 100000000LL);
+  }
   } else {
     // ------------------------------------------------ softmax / epilogue --
-    // Group w (warps 3-6: w = 0, warps 7-10: w = 1) takes the item's blocks
+    ptx::setmaxnreg_inc<C::REG_SOFTMAX>();
+    // Group w (warps 4-7: w = 0, warps 8-11: w = 1) takes the item's blocks
     // j with j % 2 == w.  Thread = one query row (TMEM lane), all 128 columns.
-    const int w = (warp - 3) >> 2;
+    const int w = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    const int gtid = threadIdx.x - 96;                 // 0..255 over both groups
+    const int gtid = threadIdx.x - 128;                // 0..255 over both groups
     const uint32_t tS = tmem + lane_base + C::COL_S + 128 * w;
     const uint32_t tP = tmem + lane_base + C::COL_P + 64 * w;
     const uint32_t tO = tmem + lane_base + C::COL_O;
@@ -739,9 +751,16 @@ template <int D, int NS, int POLY>
 cudaError_t launch_d(const TcParams& tp, int grid, cudaStream_t s) {
   using C = Cfg<D, NS, POLY>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
+  static_assert(C::REG_POOL_NEEDED <= 65536, "register split");
   cudaError_t e =
       cudaFuncSetAttribute(attn_tc_kernel<D, NS, POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
+  // The warpgroups' register increase waits for room in the block's
+  // launch-time pool: never launch a build whose pool is smaller than the split.
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D, NS, POLY>);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs * C::THREADS < C::REG_POOL_NEEDED) return cudaErrorNotSupported;
   attn_tc_kernel<D, NS, POLY><<<grid, C::THREADS, C::SMEM, s>>>(tp);
   return cudaGetLastError();
 }
