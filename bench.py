@@ -226,6 +226,63 @@ def cpu_baseline(wl, q, k, v, total_flops, budget_heads=4, qblocks=24):
 
 # ------------------------------------------------------------------ main --
 
+def selection_timing(api, q, k, wl, steps, stream, hbm_gbs):
+    """Steps 1-4 timed one stage at a time through the public C ABI on the
+    bench workload (single scheme): summarize Q, summarize K, estimate,
+    select.  L2 is flushed (a 256 MB write) before every timed call, so each
+    stage reads its inputs from HBM.  Algorithmic bytes: summarize reads one
+    [N, heads, d] tensor and writes [heads, nb, d] fp32 means; estimate reads
+    both means and writes [heads, nb, nb] fp32 probabilities (plus
+    2 nb^2 d heads FLOPs); select reads the probabilities and writes the
+    counts and the kept ids."""
+    import torch
+    sc = wl.schemes[0]
+    g = sc.as_tuple()
+    nb, heads, d = sc.nb, wl.heads, wl.d
+    esz = q.element_size()
+    qm = api.summarize(q, g)
+    km = api.summarize(k, g)
+    prob = api.estimate(qm, km)
+    cnt, idx = api.select(prob, wl.head_tau)
+    torch.cuda.synchronize()
+    kept_ids = int(cnt.sum().item())
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=q.device)
+    stages = {
+        "summarize_q": (lambda: api.summarize(q, g, out=qm), wl.N * heads * d * esz + nb * heads * d * 4, 0),
+        "summarize_k": (lambda: api.summarize(k, g, out=km), wl.N * heads * d * esz + nb * heads * d * 4, 0),
+        "estimate": (lambda: api.estimate(qm, km, out=prob), 2 * nb * heads * d * 4 + nb * nb * heads * 4,
+                     2 * nb * nb * d * heads),
+        "select": (lambda: api.select(prob, wl.head_tau, cnt=cnt, idx=idx), nb * nb * heads * 4 + nb * heads * 4
+                   + kept_ids * 4, 0),
+    }
+    out = {}
+    tot_ms, tot_bytes = 0.0, 0
+    for name, (fn, nbytes, flops) in stages.items():
+        ts = []
+        for _ in range(max(1, steps)):
+            flush.fill_(1)
+            # keep the GPU busy while the host enqueues the timed call, so the
+            # start event does not time host-side launch latency
+            torch.cuda._sleep(400000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = float(np.median(ts))
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / hbm_gbs}
+        if flops:
+            out[name]["TFLOP/s_fp32"] = flops / (ms * 1e-3) / 1e12
+        tot_ms += ms
+        tot_bytes += nbytes
+    gbs = tot_bytes / (tot_ms * 1e-3) / 1e9
+    out["total"] = {"ms": tot_ms, "bytes": tot_bytes, "GB/s": gbs, "frac_hbm": gbs / hbm_gbs,
+                    "peak_GB/s": hbm_gbs, "l2": "flushed (256 MB write) before every timed call"}
+    return out
+
+
 def workload_config(wl, tau):
     sc = wl.schemes[0]
     return {"workload": f"{wl.name}: grid {wl.T}x{wl.H}x{wl.W} ({wl.N} tokens"
@@ -398,6 +455,8 @@ def main(argv=None):
                 "frac": ach / peaks["bf16_tflops"], "traffic": None,
                 "kernel": "whole grouped step (mixed schemes)", "peak_source": f"{peaks['source']} bf16 burst"}
     extra["roofline"] = roof
+    if len(wl.schemes) == 1 and not any(wl.head_dense):
+        extra["selection"] = selection_timing(api, q, k, wl, args.steps, stream, peaks["hbm_gbs"])
     extra["ms_per_layer"] = ms
     extra["block_kept_fraction"] = float(kept_frac)
     extra["block_sparsity"] = float(1.0 - kept_frac)

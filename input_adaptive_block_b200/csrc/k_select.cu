@@ -37,7 +37,17 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __r
   const int i = (int)(row - (long long)h * nb);
   const float* prow = prob + row * nb;
   float* b = buf[warp];
-  for (int j = lane; j < nb; j += 32) b[j] = prow[j];
+  {
+    // coalesced row load, every load in flight before the first store
+    float t[NPL];
+#pragma unroll
+    for (int e = 0; e < NPL; ++e) {
+      const int j = lane + 32 * e;
+      t[e] = j < nb ? __ldg(prow + j) : 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < NPL; ++e) b[lane + 32 * e] = t[e];
+  }
   __syncwarp();
   const float tau = taus.tau[h];
   const float diag = b[i];
@@ -55,9 +65,10 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __r
     for (int bit = 29; bit >= 0; --bit) {           // p <= 1 < 2.0f = 0x40000000
       const uint32_t cand = u | (1u << bit);
       const float thr = __uint_as_float(cand);
-      float s = 0.f;
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};                // four short chains instead of one long one
 #pragma unroll
-      for (int e = 0; e < NPL; ++e) s += (v[e] >= thr) ? v[e] : 0.f;
+      for (int e = 0; e < NPL; ++e) s4[e & 3] += (v[e] >= thr) ? v[e] : 0.f;
+      float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
 #pragma unroll
       for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       if (diag + s >= tau) u = cand;

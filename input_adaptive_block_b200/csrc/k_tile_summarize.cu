@@ -45,10 +45,29 @@ __global__ void tile3d_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict
 // ------------------------------------------------------------- summarize --
 // Work unit = (block b, group of 32 16-byte chunks of a token row restricted
 // to heads [h0, h0+hc)).  One warp per unit; lane l owns chunk 32*group + l
-// and sums it over the block's valid tokens in fp32 (8-token unroll for
-// memory-level parallelism).  Units are dealt round-robin to all warps.
+// and sums it over the block's valid tokens in fp32.  The block's tokens are
+// walked in (t, y, x) order by stepping a pointer (no integer division on
+// the load path), eight loads in flight per lane.  Units are dealt
+// round-robin to all warps.
 template <bool BF16>
-__global__ void __launch_bounds__(256) summarize_kernel(const uint8_t* __restrict__ x, float* __restrict__ out,
+__device__ __forceinline__ void accumulate(float (&acc)[BF16 ? 8 : 4], const uint4& v) {
+  if (BF16) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(p[e]);
+      acc[2 * e] += f.x;
+      acc[2 * e + 1] += f.y;
+    }
+  } else {
+    const float* f = reinterpret_cast<const float*>(&v);
+#pragma unroll
+    for (int e = 0; e < (BF16 ? 8 : 4); ++e) acc[e] += f[e];
+  }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256, 5) summarize_kernel(const uint8_t* __restrict__ x, float* __restrict__ out,
                                                          Geo g, long long row_bytes, int head_off_bytes,
                                                          int chunks, int d) {
   constexpr int EPC = BF16 ? 8 : 4;  // elements per 16-byte chunk
@@ -57,6 +76,8 @@ __global__ void __launch_bounds__(256) summarize_kernel(const uint8_t* __restric
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   const int groups = (chunks + 31) / 32;
   const long long n_units = (long long)g.nb * groups;
+  const long long sy = (long long)g.W * row_bytes;     // next y row
+  const long long st = (long long)g.H * sy;            // next frame
   for (long long u = gwarp; u < n_units; u += nwarps) {
     const int b = (int)(u / groups);
     const int c = (int)(u - (long long)b * groups) * 32 + lane;
@@ -67,62 +88,45 @@ __global__ void __launch_bounds__(256) summarize_kernel(const uint8_t* __restric
 #pragma unroll
     for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
     if (c < chunks) {
-      const uint8_t* base = x + head_off_bytes + (long long)c * 16;
+      // pointer to token (t0 + tl, y0 + yl, x0 + xl); stepping x, then y, then t
+      const uint8_t* ptr = x + head_off_bytes + (long long)c * 16 +
+                           (((long long)t0 * g.H + y0) * g.W + x0) * row_bytes;
+      const long long wrap_y = sy - (long long)ew * row_bytes;
+      const long long wrap_t = st - (long long)eh * sy;
+      int xl = 0, yl = 0;
+      auto step = [&]() {
+        ptr += row_bytes;
+        if (++xl == ew) {
+          xl = 0;
+          ptr += wrap_y;
+          if (++yl == eh) {
+            yl = 0;
+            ptr += wrap_t;
+          }
+        }
+      };
       int i = 0;
       for (; i + 8 <= nvalid; i += 8) {
         uint4 v[8];
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-          const int ii = i + r;
-          const int xl = ii % ew, yl = (ii / ew) % eh, tl = ii / (ew * eh);
-          const long long tok = ((long long)(t0 + tl) * g.H + (y0 + yl)) * g.W + (x0 + xl);
-          v[r] = __ldg(reinterpret_cast<const uint4*>(base + tok * row_bytes));
+          v[r] = __ldg(reinterpret_cast<const uint4*>(ptr));
+          step();
         }
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          if (BF16) {
-            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[r]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float2 f = __bfloat1622float2(p[e]);
-              acc[2 * e] += f.x;
-              acc[2 * e + 1] += f.y;
-            }
-          } else {
-            const float* f = reinterpret_cast<const float*>(&v[r]);
-#pragma unroll
-            for (int e = 0; e < EPC; ++e) acc[e] += f[e];
-          }
-        }
+        for (int r = 0; r < 8; ++r) accumulate<BF16>(acc, v[r]);
       }
       for (; i < nvalid; ++i) {
-        const int xl = i % ew, yl = (i / ew) % eh, tl = i / (ew * eh);
-        const long long tok = ((long long)(t0 + tl) * g.H + (y0 + yl)) * g.W + (x0 + xl);
-        uint4 v = __ldg(reinterpret_cast<const uint4*>(base + tok * row_bytes));
-        if (BF16) {
-          const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float2 f = __bfloat1622float2(p[e]);
-            acc[2 * e] += f.x;
-            acc[2 * e + 1] += f.y;
-          }
-        } else {
-          const float* f = reinterpret_cast<const float*>(&v);
-#pragma unroll
-          for (int e = 0; e < EPC; ++e) acc[e] += f[e];
-        }
+        accumulate<BF16>(acc, __ldg(reinterpret_cast<const uint4*>(ptr)));
+        step();
       }
       const float inv = 1.0f / (float)nvalid;
       const int e0 = c * EPC;             // element index within the head-range row
       const int h = e0 / d, dd = e0 - h * d;
       float* o = out + ((long long)h * g.nb + b) * d + dd;
-      if (BF16) {
-        reinterpret_cast<float4*>(o)[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+      reinterpret_cast<float4*>(o)[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+      if (BF16)
         reinterpret_cast<float4*>(o)[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
-      } else {
-        reinterpret_cast<float4*>(o)[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-      }
     }
   }
 }
@@ -145,7 +149,7 @@ cudaError_t launch_summarize(const void* x, float* out, const Geo& g, int heads_
   const int groups = (chunks + 31) / 32;
   const long long units = (long long)g.nb * groups;
   long long blocks = (units + 7) / 8;                  // 8 warps per CTA
-  const long long cap = 2LL * num_sms();               // 16 resident warps per SM
+  const long long cap = 5LL * num_sms();               // all resident: 40 warps per SM
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   if (dt == SPADE_BF16)
