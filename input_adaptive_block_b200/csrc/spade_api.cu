@@ -146,6 +146,18 @@ spade_status plan_group(const spade_geom* schemes, int n_schemes, const spade_he
   return SPADE_OK;
 }
 
+// Step 3: the tensor-core estimator (split-precision TF32); the FMA-pipe
+// kernel only when the tensor-map encoder is unavailable.
+cudaError_t run_estimate(const float* qm, const float* km, float* prob, int heads, int nb, int d, int* status,
+                         cudaStream_t s) {
+  cudaError_t e = launch_estimate_tc(qm, km, prob, heads, nb, d, status, s);
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    e = launch_estimate(qm, km, prob, heads, nb, d, s);
+  }
+  return e;
+}
+
 spade_status run_attention(AttnArgs& a, cudaStream_t s) {
   a.status = status_ptr();
   if (!a.status) return fail(SPADE_ERR_CUDA, "device status word unavailable");
@@ -266,7 +278,9 @@ spade_status spade_estimate(const float* qmean, const float* kmean, float* prob,
   if (nb < 1) return fail(SPADE_ERR_INVALID, "nb=%d", nb);
   if (nb > SPADE_ESTIMATE_MAX_NB) return fail(SPADE_ERR_UNSUPPORTED, "nb=%d above %d", nb, SPADE_ESTIMATE_MAX_NB);
   if (d != 64 && d != 128) return fail(SPADE_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", d);
-  cudaError_t e = launch_estimate(qmean, kmean, prob, heads, nb, d, as_cuda(stream));
+  int* st = status_ptr();
+  if (!st) return fail(SPADE_ERR_CUDA, "device status word unavailable");
+  cudaError_t e = run_estimate(qmean, kmean, prob, heads, nb, d, st, as_cuda(stream));
   return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "estimate");
 }
 
@@ -418,7 +432,9 @@ spade_status spade_grouped_attn(const void* q, const void* k, const void* v, voi
       i = j;
     }
     float* prob = reinterpret_cast<float*>(ws + L.prob[sc]);
-    cudaError_t e = launch_estimate(qm, km, prob, hs, g.nb, d, s);
+    int* st = status_ptr();
+    if (!st) return fail(SPADE_ERR_CUDA, "device status word unavailable");
+    cudaError_t e = run_estimate(qm, km, prob, hs, g.nb, d, st, s);
     if (e != cudaSuccess) return cuda_fail(e, "estimate");
     std::vector<float> taus(hs);
     for (int i = 0; i < hs; ++i) taus[i] = table[hl[i]].tau;

@@ -81,6 +81,8 @@ cudaError_t launch_tile3d(const void* x, void* xt, const Geo& g, int heads, int 
                           cudaStream_t s);
 cudaError_t launch_summarize(const void* x, float* out, const Geo& g, int heads_total, int h0, int hc, int d,
                              spade_dtype dt, cudaStream_t s);
+cudaError_t launch_estimate_tc(const float* qm, const float* km, float* prob, int heads, int nb, int d, int* status,
+                               cudaStream_t s);
 cudaError_t launch_estimate(const float* qm, const float* km, float* prob, int heads, int nb, int d,
                             cudaStream_t s);
 cudaError_t launch_select(const float* prob, const float* tau_host, int* cnt, int* idx, int heads, int nb,
