@@ -51,6 +51,7 @@ __all__ = [
     "block_tokens", "valid_counts", "tile3d", "untile3d", "summarize", "estimate",
     "select_row", "select", "selection_margin", "attention_rows", "block_sparse_attention",
     "dense_attention", "pipeline", "kept_token_pairs",
+    "block_sics", "sics", "choose_schemes",
 ]
 
 
@@ -291,6 +292,61 @@ def kept_token_pairs(head_geom, head_kept, text_tokens: int = 0,
             else:
                 total += int(vc[i]) * (int(vc[list(head_kept[h][i])].sum()) + text_tokens)
     return total
+
+
+# ---------------------------------------------------------------------------
+# Scheme generation: Sum of Intra-block Cosine Similarities (SICS)
+# ---------------------------------------------------------------------------
+# Technical summary, Methodology 2 "Scheme Generation", Aggregation
+# Evaluation: every blocking candidate is scored by the sum of the cosine
+# similarities between the embeddings inside each block (tightly clustered
+# blocks score high); Policy Application: each head takes the candidate with
+# the highest score.  Readings (the pages give no formula): the embeddings
+# are the head's Q and K tokens, scored separately and added; the sum runs
+# over ordered pairs (i, j) of valid tokens of a block, i = j included (that
+# adds N to every candidate alike, so the choice is unaffected); a zero
+# vector has cosine 0 with everything; ties go to the lower candidate index.
+
+def block_sics(xb: np.ndarray) -> float:
+    """sum_{i, j} cos(x_i, x_j) over the rows of xb, by the plain pairwise
+    definition: O(n^2 d)."""
+    x = np.asarray(xb, dtype=np.float64)
+    nrm = np.sqrt(np.sum(x * x, axis=1))
+    total = 0.0
+    for i in range(x.shape[0]):
+        for j in range(x.shape[0]):
+            if nrm[i] > 0.0 and nrm[j] > 0.0:
+                total += float(np.dot(x[i], x[j]) / (nrm[i] * nrm[j]))
+    return total
+
+
+def sics(x: np.ndarray, geom: Sequence[int]) -> np.ndarray:
+    """[heads] SICS of one tensor x [N, heads, d] under one blocking scheme:
+    the sum over its blocks of block_sics of the block's valid tokens."""
+    T, H, W, bt, bh, bw = (int(g) for g in geom)
+    heads = x.shape[1]
+    out = np.zeros(heads, dtype=np.float64)
+    for ids, _slots in block_tokens(T, H, W, bt, bh, bw):
+        for h in range(heads):
+            out[h] += block_sics(x[ids, h, :])
+    return out
+
+
+def choose_schemes(q: np.ndarray, k: np.ndarray, candidates: Sequence[Sequence[int]]):
+    """Per head: the SICS of every candidate (Q plus K) and the index of the
+    best one.  Returns (scores [heads, n_candidates], choice [heads])."""
+    heads = q.shape[1]
+    scores = np.zeros((heads, len(candidates)), dtype=np.float64)
+    for c, geom in enumerate(candidates):
+        scores[:, c] = sics(q, geom) + sics(k, geom)
+    choice = np.zeros(heads, dtype=np.int64)
+    for h in range(heads):
+        best = 0
+        for c in range(1, len(candidates)):
+            if scores[h, c] > scores[h, best]:
+                best = c
+        choice[h] = best
+    return scores, choice
 
 
 # ---------------------------------------------------------------------------
