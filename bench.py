@@ -283,6 +283,36 @@ def selection_timing(api, q, k, wl, steps, stream, hbm_gbs):
     return out
 
 
+def sics_timing(api, q, k, wl, steps, stream, hbm_gbs):
+    """Scheme generation (spade_sics) on the bench layer with the three
+    candidates of the mixed head-wise policy (2x8x8, 1x8x16, 8x4x4): one pass
+    over Q and K per candidate, L2 flushed before each timed call.
+    Algorithmic bytes: n_candidates x (Q + K) read, scores written."""
+    import torch
+    T, H, W = wl.T, wl.H, wl.W
+    cands = [(T, H, W, 2, 8, 8), (T, H, W, 1, 8, 16), (T, H, W, 8, 4, 4)]
+    ws = torch.empty(api.sics_workspace_bytes(cands, wl.heads), dtype=torch.uint8, device=q.device)
+    api.sics(q, k, cands, workspace=ws)
+    torch.cuda.synchronize()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=q.device)
+    ts = []
+    for _ in range(max(1, steps)):
+        flush.fill_(1)
+        torch.cuda._sleep(400000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        scores, choice = api.sics(q, k, cands, workspace=ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ms = float(np.median(ts))
+    nbytes = len(cands) * 2 * wl.N * wl.heads * wl.d * q.element_size()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    picks = np.bincount(choice.cpu().numpy(), minlength=len(cands)).tolist()
+    return {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / hbm_gbs, "candidates": ["2x8x8", "1x8x16", "8x4x4"],
+            "heads_per_candidate": picks, "l2": "flushed (256 MB write) before every timed call"}
+
+
 def workload_config(wl, tau):
     sc = wl.schemes[0]
     return {"workload": f"{wl.name}: grid {wl.T}x{wl.H}x{wl.W} ({wl.N} tokens"
@@ -457,6 +487,8 @@ def main(argv=None):
     extra["roofline"] = roof
     if len(wl.schemes) == 1 and not any(wl.head_dense):
         extra["selection"] = selection_timing(api, q, k, wl, args.steps, stream, peaks["hbm_gbs"])
+        if wl.text_tokens == 0 and wl.d == 128:
+            extra["scheme_generation"] = sics_timing(api, q, k, wl, args.steps, stream, peaks["hbm_gbs"])
     extra["ms_per_layer"] = ms
     extra["block_kept_fraction"] = float(kept_frac)
     extra["block_sparsity"] = float(1.0 - kept_frac)

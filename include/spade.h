@@ -183,6 +183,31 @@ spade_status spade_grouped_head_lists(const spade_geom* schemes, int n_schemes,
                                       int text_tokens, int head,
                                       int64_t* cnt_offset, int64_t* idx_offset);
 
+/* ---- scheme generation: Sum of Intra-block Cosine Similarities -----------
+ * Technical summary, Methodology 2 "Scheme Generation": every blocking
+ * candidate is scored by the sum of the cosine similarities between the
+ * embeddings inside each of its blocks (Aggregation Evaluation, in the
+ * O(BS * d) online form), and each head takes the candidate with the
+ * highest score (Policy Application); the result fills the per-head scheme
+ * table of spade_grouped_attn.  Score of head h under candidate c:
+ *   sum over blocks b of sum_{i,j valid in b} cos(q_i, q_j) + cos(k_i, k_j)
+ * (ordered pairs, i = j included; a zero vector counts 0), evaluated as
+ * || sum_i q_i/||q_i|| ||^2 + || sum_i k_i/||k_i|| ||^2 per block.
+ * q, k      : device [N, heads, d] in dt, token order (text tokens, if any,
+ *             follow the video tokens and are not scored).
+ * candidates: n_candidates (1..4) geometries over the same T*H*W = N.
+ * scores    : device float [heads, n_candidates] (written).
+ * choice    : device int32 [heads]: index of the best candidate, ties to the
+ *             lower index (written).
+ * workspace : device scratch of spade_sics_workspace_bytes() bytes (one
+ *             float per head, block and candidate); sums run in a fixed
+ *             order, so results are deterministic.
+ * Supported: d in {64, 128}, dt bf16 or f32, heads <= 1024. */
+size_t spade_sics_workspace_bytes(const spade_geom* candidates, int n_candidates, int heads);
+spade_status spade_sics(const void* q, const void* k, const spade_geom* candidates, int n_candidates,
+                        int heads, int d, spade_dtype dt, float* scores, int* choice,
+                        void* workspace, size_t ws_bytes, spade_stream_t stream);
+
 /* ---- status ---------------------------------------------------------------
  * spade_last_device_status synchronises `stream`, returns the latched device
  * status (SPADE_OK or SPADE_ERR_TIMEOUT) and clears it. */

@@ -43,6 +43,9 @@ SIGNATURES = {
                                    c_size_t, c_void_p]),
     "spade_grouped_head_lists": (c_int, [POINTER(SpadeGeom), c_int, POINTER(SpadeHeadScheme), c_int,
                                          c_int, c_int, c_int, POINTER(c_int64), POINTER(c_int64)]),
+    "spade_sics_workspace_bytes": (c_size_t, [POINTER(SpadeGeom), c_int, c_int]),
+    "spade_sics": (c_int, [c_void_p, c_void_p, POINTER(SpadeGeom), c_int, c_int, c_int, c_int, c_void_p, c_void_p,
+                           c_void_p, c_size_t, c_void_p]),
     "spade_last_device_status": (c_int, [c_void_p]),
     "spade_status_string": (ctypes.c_char_p, [c_int]),
     "spade_last_error_message": (ctypes.c_char_p, []),

@@ -17,7 +17,7 @@ from ._lib import SpadeGeom, SpadeHeadScheme, check
 __all__ = [
     "geom", "dtype_code", "tile3d", "summarize", "estimate", "select", "attn_workspace_bytes",
     "block_sparse_attn", "block_sparse_attn_noalloc", "grouped_workspace_bytes", "grouped_attn", "grouped_head_lists",
-    "last_device_status", "selftest_bounded_wait", "num_blocks",
+    "last_device_status", "selftest_bounded_wait", "num_blocks", "sics_workspace_bytes", "sics",
 ]
 
 
@@ -175,6 +175,29 @@ def grouped_head_lists(schemes, table, d: int, text_tokens: int, head: int) -> T
     check(_lib.load().spade_grouped_head_lists(gs, len(schemes), rows, len(table), d, text_tokens, head,
                                                ctypes.byref(co), ctypes.byref(io)), "spade_grouped_head_lists")
     return co.value, io.value
+
+
+def sics_workspace_bytes(candidates, heads: int) -> int:
+    gs = (SpadeGeom * len(candidates))(*[geom(c) for c in candidates])
+    return int(_lib.load().spade_sics_workspace_bytes(gs, len(candidates), heads))
+
+
+def sics(q: torch.Tensor, k: torch.Tensor, candidates, workspace: Optional[torch.Tensor] = None,
+         stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Scheme generation: per head, the SICS of every candidate blocking
+    scheme (Q plus K) and the index of the best one.  Returns (scores
+    [heads, n_candidates] float32, choice [heads] int32), both on the device."""
+    heads, d = q.shape[1], q.shape[2]
+    gs = (SpadeGeom * len(candidates))(*[geom(c) for c in candidates])
+    scores = torch.empty(heads, len(candidates), dtype=torch.float32, device=q.device)
+    choice = torch.empty(heads, dtype=torch.int32, device=q.device)
+    if workspace is None:
+        need = int(_lib.load().spade_sics_workspace_bytes(gs, len(candidates), heads))
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    check(_lib.load().spade_sics(_dev(q, "q"), _dev(k, "k"), gs, len(candidates), heads, d, dtype_code(q.dtype),
+                                 _dev(scores, "scores"), _dev(choice, "choice"), _dev(workspace, "workspace"),
+                                 workspace.numel(), _stream(stream)), "spade_sics")
+    return scores, choice
 
 
 def last_device_status(stream=None) -> int:

@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build", "spade")
 LIB = os.path.join(PKG, "libspade.so")
 
-SOURCES = ["spade_api.cu", "k_tile_summarize.cu", "k_estimate.cu", "k_estimate_tc.cu", "k_select.cu",
+SOURCES = ["spade_api.cu", "k_tile_summarize.cu", "k_estimate.cu", "k_estimate_tc.cu", "k_select.cu", "k_sics.cu",
            "k_attn_simt.cu", "k_attn_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]

@@ -385,6 +385,39 @@ size_t spade_grouped_workspace_bytes(const spade_geom* schemes, int n_schemes, c
   return L.total;
 }
 
+size_t spade_sics_workspace_bytes(const spade_geom* candidates, int n_candidates, int heads) {
+  if (!candidates || n_candidates < 1 || n_candidates > SPADE_MAX_SCHEMES || heads < 1) return 0;
+  Geo g[SPADE_MAX_SCHEMES];
+  for (int c = 0; c < n_candidates; ++c) g[c] = make_geo(candidates[c]);
+  return sics_workspace_floats(g, n_candidates, heads) * sizeof(float);
+}
+
+spade_status spade_sics(const void* q, const void* k, const spade_geom* candidates, int n_candidates, int heads,
+                        int d, spade_dtype dt, float* scores, int* choice, void* workspace, size_t ws_bytes,
+                        spade_stream_t stream) {
+  if (!q || !k || !candidates || !scores || !choice || !workspace) return fail(SPADE_ERR_INVALID, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(workspace))
+    return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  if (n_candidates < 1 || n_candidates > SPADE_MAX_SCHEMES)
+    return fail(SPADE_ERR_INVALID, "n_candidates=%d (1..%d)", n_candidates, SPADE_MAX_SCHEMES);
+  if (heads < 1 || heads > 1024) return fail(SPADE_ERR_INVALID, "heads=%d", heads);
+  spade_status st = check_d_dt(d, dt);
+  if (st != SPADE_OK) return st;
+  Geo g[SPADE_MAX_SCHEMES];
+  for (int c = 0; c < n_candidates; ++c) {
+    if ((st = check_geom(candidates[c])) != SPADE_OK) return st;
+    if ((long long)candidates[c].T * candidates[c].H * candidates[c].W !=
+        (long long)candidates[0].T * candidates[0].H * candidates[0].W)
+      return fail(SPADE_ERR_INVALID, "candidate %d covers a different number of tokens", c);
+    g[c] = make_geo(candidates[c]);
+  }
+  const size_t need = sics_workspace_floats(g, n_candidates, heads) * sizeof(float);
+  if (ws_bytes < need) return fail(SPADE_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  cudaError_t e = launch_sics(q, k, g, n_candidates, heads, d, dt, static_cast<float*>(workspace), scores, choice,
+                              as_cuda(stream));
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "sics");
+}
+
 spade_status spade_grouped_head_lists(const spade_geom* schemes, int n_schemes, const spade_head_scheme* table,
                                       int heads, int d, int text_tokens, int head, int64_t* cnt_offset,
                                       int64_t* idx_offset) {

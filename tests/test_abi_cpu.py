@@ -106,3 +106,24 @@ def test_attn_workspace_bytes():
     assert lib.spade_attn_workspace_bytes(g, 40, 128, 0) >= 40 * 660 * 4
     assert lib.spade_attn_workspace_bytes(g, 40, 128, 256) >= 40 * 662 * 4
     assert lib.spade_attn_workspace_bytes(SpadeGeom(0, 1, 1, 1, 1, 1), 1, 128, 0) == 0
+
+
+def test_sics_host_validation():
+    lib = _lib.load()
+    g1 = SpadeGeom(21, 45, 80, 2, 8, 8)
+    cands = (SpadeGeom * 3)(g1, SpadeGeom(21, 45, 80, 1, 8, 16), SpadeGeom(21, 45, 80, 8, 4, 4))
+    need = lib.spade_sics_workspace_bytes(cands, 3, 40)
+    assert need == 4 * 40 * (660 + 630 + 720)
+    assert lib.spade_sics_workspace_bytes(cands, 0, 40) == 0
+    fake = ctypes.c_void_p(1 << 20)                 # never dereferenced: validation fails first
+    args = lambda **kw: dict(dict(q=fake, k=fake, c=cands, n=3, h=40, d=128, dt=1, s=fake, ch=fake, ws=fake,
+                                  wsb=need), **kw)
+    call = lambda a: lib.spade_sics(a["q"], a["k"], a["c"], a["n"], a["h"], a["d"], a["dt"], a["s"], a["ch"],
+                                    a["ws"], a["wsb"], None)
+    assert call(args(q=None)) == _lib.SPADE_ERR_INVALID
+    assert call(args(n=0)) == _lib.SPADE_ERR_INVALID
+    assert call(args(d=96)) == _lib.SPADE_ERR_UNSUPPORTED
+    assert call(args(wsb=16)) == _lib.SPADE_ERR_WORKSPACE
+    other = (SpadeGeom * 2)(g1, SpadeGeom(21, 45, 81, 2, 8, 8))
+    assert call(args(c=other, n=2)) == _lib.SPADE_ERR_INVALID
+    assert b"different number of tokens" in lib.spade_last_error_message()
