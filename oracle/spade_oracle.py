@@ -118,13 +118,24 @@ def untile3d(xt: np.ndarray, geom: Sequence[int]) -> np.ndarray:
 # 2. Summarizer: block mean over valid tokens
 # ---------------------------------------------------------------------------
 
-def summarize(x: np.ndarray, geom: Sequence[int]) -> np.ndarray:
-    """Mean of each block's valid tokens: [N, heads, d] -> [heads, nb, d]."""
+def summarize(x: np.ndarray, geom: Sequence[int], mode: str = "mean") -> np.ndarray:
+    """Reduce each block's valid tokens: [N, heads, d] -> [heads, nb, d].
+    mode "mean" (the instance the estimator is specified with), or the other
+    reduces the Summarizer names, "max" / "min" (elementwise over the block's
+    valid tokens; padding never takes part)."""
     blocks = block_tokens(*geom)
     heads, d = x.shape[1], x.shape[2]
     out = np.zeros((heads, len(blocks), d), dtype=np.float64)
     for b, (toks, _) in enumerate(blocks):
-        out[:, b, :] = x[toks].astype(np.float64).sum(axis=0) / len(toks)
+        xb = x[toks].astype(np.float64)
+        if mode == "mean":
+            out[:, b, :] = xb.sum(axis=0) / len(toks)
+        elif mode == "max":
+            out[:, b, :] = xb.max(axis=0)
+        elif mode == "min":
+            out[:, b, :] = xb.min(axis=0)
+        else:
+            raise ValueError(mode)
     return out
 
 
@@ -358,11 +369,12 @@ def pipeline(q: np.ndarray, k: np.ndarray, v: np.ndarray,
              head_tau: Sequence[float], head_dense: Sequence[bool],
              text_tokens: int = 0,
              q_blocks: Optional[Dict[int, Sequence[int]]] = None,
-             kept_override: Optional[Dict[int, Sequence[Sequence[int]]]] = None) -> dict:
-    """Steps 1-5 for every head.  Returns the per-scheme means and
+             kept_override: Optional[Dict[int, Sequence[Sequence[int]]]] = None,
+             summary: Tuple[str, str] = ("mean", "mean")) -> dict:
+    """Steps 1-5 for every head.  Returns the per-scheme summaries and
     probabilities, the kept lists and the output.  kept_override replaces the
     oracle's own selection for the given heads (used to evaluate attention
-    under another implementation's mask)."""
+    under another implementation's mask); summary picks the Q and K reduces."""
     heads = q.shape[1]
     N = q.shape[0] - text_tokens
     head_geom = [tuple(schemes[head_scheme[h]]) for h in range(heads)]
@@ -371,8 +383,8 @@ def pipeline(q: np.ndarray, k: np.ndarray, v: np.ndarray,
         hs = [h for h in range(heads) if head_scheme[h] == s_id and not head_dense[h]]
         if not hs:
             continue
-        qm = summarize(q[:N, hs], geom)
-        km = summarize(k[:N, hs], geom)
+        qm = summarize(q[:N, hs], geom, summary[0])
+        km = summarize(k[:N, hs], geom, summary[1])
         P = estimate(qm, km)
         res["qmean"][s_id], res["kmean"][s_id], res["prob"][s_id] = qm, km, P
         for n, h in enumerate(hs):

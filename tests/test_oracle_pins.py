@@ -332,3 +332,34 @@ def test_planted_mistakes_are_caught(golden_dir, monkeypatch):
     blocks = O.block_tokens(*geom)
     padded_mean = np.array([len(t) / 32.0 for t, _ in blocks])
     assert not np.allclose(padded_mean, O.summarize(xx, geom)[0, :, 0])
+
+
+# ---- Summarizer variants (max / min reduces) ----
+
+def test_summarize_max_min_properties():
+    """max/min are attained by a valid token of the block, bound every valid
+    token and bracket the mean; padding never takes part (an all-negative
+    ragged input would show a padded zero as the max)."""
+    rng = np.random.default_rng(11)
+    geom = (3, 5, 7, 2, 4, 4)                       # ragged in every dimension
+    x = -np.abs(rng.standard_normal((3 * 5 * 7, 2, 6))) - 0.1
+    mx, mn, me = (O.summarize(x, geom, m) for m in ("max", "min", "mean"))
+    for b, (toks, _) in enumerate(O.block_tokens(*geom)):
+        xb = x[toks]                                  # [n, heads, d]
+        for h in range(2):
+            for c in range(6):
+                col = xb[:, h, c]
+                assert mx[h, b, c] in set(col.tolist()) and mn[h, b, c] in set(col.tolist())
+                assert (col <= mx[h, b, c]).all() and (col >= mn[h, b, c]).all()
+                assert mn[h, b, c] <= me[h, b, c] <= mx[h, b, c]
+    assert (mx < 0).all()
+
+
+def test_summarize_modes_agree_on_constant_blocks():
+    geom = (4, 4, 4, 2, 2, 2)
+    vals = np.arange(8, dtype=np.float64)
+    x = np.zeros((64, 1, 3))
+    for b, (toks, _) in enumerate(O.block_tokens(*geom)):
+        x[toks] = vals[b]
+    for m in ("mean", "max", "min"):
+        assert np.allclose(O.summarize(x, geom, m)[0, :, 0], vals)
