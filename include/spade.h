@@ -63,6 +63,10 @@ typedef enum {
 
 typedef enum { SPADE_F32 = 0, SPADE_BF16 = 1 } spade_dtype;
 
+/* Summarizer reduce of a Q/K block (Methodology 1, "Summarizer & Estimator
+ * Expressions": max / min / mean), over the block's valid tokens. */
+typedef enum { SPADE_SUM_MEAN = 0, SPADE_SUM_MAX = 1, SPADE_SUM_MIN = 2 } spade_summary;
+
 /* One blocking scheme: the (T,H,W) latent grid cut into (bt,bh,bw) boxes.
  * A dense head may use the flat scheme {1,1,N, 1,1,128}. */
 typedef struct { int32_t T, H, W, bt, bh, bw; } spade_geom;
@@ -90,6 +94,13 @@ spade_status spade_tile3d(const void* x, void* xt, spade_geom g, int heads, int 
  *         (accumulated in float32). */
 spade_status spade_summarize(const void* x, float* xmean, spade_geom g, int heads, int d,
                              spade_dtype dt, spade_stream_t stream);
+
+/* The same pass with another of the Summarizer's reduces: mode
+ * SPADE_SUM_MAX / SPADE_SUM_MIN give the elementwise max / min over each
+ * block's valid tokens (exact: no rounding), SPADE_SUM_MEAN is
+ * spade_summarize. */
+spade_status spade_summarize_mode(const void* x, float* out, spade_geom g, int heads, int d,
+                                  spade_dtype dt, spade_summary mode, spade_stream_t stream);
 
 /* ---- step 3: Estimator ---------------------------------------------------
  * Methodology 1, "Summarizer & Estimator Expressions" (inter-block importance).
@@ -174,6 +185,16 @@ spade_status spade_grouped_attn(const void* q, const void* k, const void* v, voi
                                 const spade_head_scheme* table, int heads, int d,
                                 int text_tokens, spade_dtype dt,
                                 void* workspace, size_t ws_bytes, spade_stream_t stream);
+
+/* spade_grouped_attn with the Summarizer reduce chosen for Q and for K
+ * (the estimator then scores the pooled Q and K summaries as usual);
+ * spade_grouped_attn is this call with SPADE_SUM_MEAN for both. */
+spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, void* out,
+                                   const spade_geom* schemes, int n_schemes,
+                                   const spade_head_scheme* table, int heads, int d,
+                                   int text_tokens, spade_dtype dt,
+                                   spade_summary q_summary, spade_summary k_summary,
+                                   void* workspace, size_t ws_bytes, spade_stream_t stream);
 
 /* Where, inside a grouped workspace, head `head`'s kept lists live (byte
  * offsets of its int32 cnt [nb] and idx [nb, nb] arrays); -1 for dense heads.

@@ -43,6 +43,10 @@ SIGNATURES = {
                                    c_size_t, c_void_p]),
     "spade_grouped_head_lists": (c_int, [POINTER(SpadeGeom), c_int, POINTER(SpadeHeadScheme), c_int,
                                          c_int, c_int, c_int, POINTER(c_int64), POINTER(c_int64)]),
+    "spade_summarize_mode": (c_int, [c_void_p, c_void_p, SpadeGeom, c_int, c_int, c_int, c_int, c_void_p]),
+    "spade_grouped_attn_ex": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SpadeGeom), c_int,
+                                      POINTER(SpadeHeadScheme), c_int, c_int, c_int, c_int, c_int, c_int,
+                                      c_void_p, c_size_t, c_void_p]),
     "spade_sics_workspace_bytes": (c_size_t, [POINTER(SpadeGeom), c_int, c_int]),
     "spade_sics": (c_int, [c_void_p, c_void_p, POINTER(SpadeGeom), c_int, c_int, c_int, c_int, c_void_p, c_void_p,
                            c_void_p, c_size_t, c_void_p]),

@@ -64,13 +64,23 @@ def tile3d(x: torch.Tensor, g, out: Optional[torch.Tensor] = None, stream=None) 
     return out
 
 
-def summarize(x: torch.Tensor, g, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+SUMMARY = {"mean": 0, "max": 1, "min": 2}
+
+
+def summarize(x: torch.Tensor, g, out: Optional[torch.Tensor] = None, stream=None,
+              mode: str = "mean") -> torch.Tensor:
+    """Block summaries [heads, nb, d] float32: mean (default), max or min
+    over each block's valid tokens."""
     gg = geom(g)
     heads, d = x.shape[1], x.shape[2]
     if out is None:
         out = torch.empty(heads, num_blocks(gg), d, dtype=torch.float32, device=x.device)
-    check(_lib.load().spade_summarize(_dev(x, "x"), _dev(out, "xmean"), gg, heads, d, dtype_code(x.dtype),
-                                      _stream(stream)), "spade_summarize")
+    if mode == "mean":
+        check(_lib.load().spade_summarize(_dev(x, "x"), _dev(out, "xmean"), gg, heads, d, dtype_code(x.dtype),
+                                          _stream(stream)), "spade_summarize")
+    else:
+        check(_lib.load().spade_summarize_mode(_dev(x, "x"), _dev(out, "out"), gg, heads, d, dtype_code(x.dtype),
+                                               SUMMARY[mode], _stream(stream)), "spade_summarize_mode")
     return out
 
 
@@ -152,8 +162,9 @@ def grouped_workspace_bytes(schemes, table, d: int, text_tokens: int = 0) -> int
 
 def grouped_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, schemes, table, text_tokens: int = 0,
                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                 stream=None) -> torch.Tensor:
-    """table: per head (scheme index, tau, dense)."""
+                 stream=None, summary=("mean", "mean")) -> torch.Tensor:
+    """table: per head (scheme index, tau, dense); summary: the Q and K
+    Summarizer reduces ("mean", "max" or "min")."""
     heads, d = q.shape[1], q.shape[2]
     gs, rows = _tables(schemes, table)
     if out is None:
@@ -161,10 +172,16 @@ def grouped_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, schemes, tab
     if workspace is None:
         need = int(_lib.load().spade_grouped_workspace_bytes(gs, len(schemes), rows, heads, d, text_tokens))
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    check(_lib.load().spade_grouped_attn(
-        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), gs, len(schemes), rows, heads, d,
-        text_tokens, dtype_code(q.dtype), _dev(workspace, "workspace"), workspace.numel(), _stream(stream)),
-        "spade_grouped_attn")
+    if tuple(summary) == ("mean", "mean"):
+        check(_lib.load().spade_grouped_attn(
+            _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), gs, len(schemes), rows, heads, d,
+            text_tokens, dtype_code(q.dtype), _dev(workspace, "workspace"), workspace.numel(), _stream(stream)),
+            "spade_grouped_attn")
+    else:
+        check(_lib.load().spade_grouped_attn_ex(
+            _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), gs, len(schemes), rows, heads, d,
+            text_tokens, dtype_code(q.dtype), SUMMARY[summary[0]], SUMMARY[summary[1]],
+            _dev(workspace, "workspace"), workspace.numel(), _stream(stream)), "spade_grouped_attn_ex")
     return out
 
 

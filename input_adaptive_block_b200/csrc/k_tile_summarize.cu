@@ -49,24 +49,31 @@ __global__ void tile3d_kernel(const uint8_t* __restrict__ x, uint8_t* __restrict
 // walked in (t, y, x) order by stepping a pointer (no integer division on
 // the load path), eight loads in flight per lane.  Units are dealt
 // round-robin to all warps.
-template <bool BF16>
+// MODE: 0 mean (sum, divided at the end), 1 max, 2 min -- the Summarizer's
+// reduces (Methodology 1 names max / min / mean).
+template <int MODE>
+__device__ __forceinline__ float combine(float a, float v) {
+  return MODE == 0 ? a + v : (MODE == 1 ? fmaxf(a, v) : fminf(a, v));
+}
+
+template <bool BF16, int MODE>
 __device__ __forceinline__ void accumulate(float (&acc)[BF16 ? 8 : 4], const uint4& v) {
   if (BF16) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 f = __bfloat1622float2(p[e]);
-      acc[2 * e] += f.x;
-      acc[2 * e + 1] += f.y;
+      acc[2 * e] = combine<MODE>(acc[2 * e], f.x);
+      acc[2 * e + 1] = combine<MODE>(acc[2 * e + 1], f.y);
     }
   } else {
     const float* f = reinterpret_cast<const float*>(&v);
 #pragma unroll
-    for (int e = 0; e < (BF16 ? 8 : 4); ++e) acc[e] += f[e];
+    for (int e = 0; e < (BF16 ? 8 : 4); ++e) acc[e] = combine<MODE>(acc[e], f[e]);
   }
 }
 
-template <bool BF16>
+template <bool BF16, int MODE>
 __global__ void __launch_bounds__(256, 5) summarize_kernel(const uint8_t* __restrict__ x, float* __restrict__ out,
                                                          Geo g, long long row_bytes, int head_off_bytes,
                                                          int chunks, int d) {
@@ -86,7 +93,7 @@ __global__ void __launch_bounds__(256, 5) summarize_kernel(const uint8_t* __rest
     const int nvalid = et * eh * ew;
     float acc[EPC];
 #pragma unroll
-    for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+    for (int e = 0; e < EPC; ++e) acc[e] = MODE == 0 ? 0.f : (MODE == 1 ? -INFINITY : INFINITY);
     if (c < chunks) {
       // pointer to token (t0 + tl, y0 + yl, x0 + xl); stepping x, then y, then t
       const uint8_t* ptr = x + head_off_bytes + (long long)c * 16 +
@@ -114,13 +121,13 @@ __global__ void __launch_bounds__(256, 5) summarize_kernel(const uint8_t* __rest
           step();
         }
 #pragma unroll
-        for (int r = 0; r < 8; ++r) accumulate<BF16>(acc, v[r]);
+        for (int r = 0; r < 8; ++r) accumulate<BF16, MODE>(acc, v[r]);
       }
       for (; i < nvalid; ++i) {
-        accumulate<BF16>(acc, __ldg(reinterpret_cast<const uint4*>(ptr)));
+        accumulate<BF16, MODE>(acc, __ldg(reinterpret_cast<const uint4*>(ptr)));
         step();
       }
-      const float inv = 1.0f / (float)nvalid;
+      const float inv = MODE == 0 ? 1.0f / (float)nvalid : 1.0f;
       const int e0 = c * EPC;             // element index within the head-range row
       const int h = e0 / d, dd = e0 - h * d;
       float* o = out + ((long long)h * g.nb + b) * d + dd;
@@ -141,8 +148,9 @@ cudaError_t launch_tile3d(const void* x, void* xt, const Geo& g, int heads, int 
   return cudaGetLastError();
 }
 
-cudaError_t launch_summarize(const void* x, float* out, const Geo& g, int heads_total, int h0, int hc, int d,
-                             spade_dtype dt, cudaStream_t s) {
+template <int MODE>
+cudaError_t launch_summarize_m(const void* x, float* out, const Geo& g, int heads_total, int h0, int hc, int d,
+                               spade_dtype dt, cudaStream_t s) {
   const int esz = dt == SPADE_BF16 ? 2 : 4;
   const long long row_bytes = (long long)heads_total * d * esz;
   const int chunks = hc * d * esz / 16;
@@ -153,12 +161,19 @@ cudaError_t launch_summarize(const void* x, float* out, const Geo& g, int heads_
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   if (dt == SPADE_BF16)
-    summarize_kernel<true><<<(int)blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), out, g, row_bytes,
-                                                        h0 * d * esz, chunks, d);
+    summarize_kernel<true, MODE><<<(int)blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), out, g, row_bytes,
+                                                              h0 * d * esz, chunks, d);
   else
-    summarize_kernel<false><<<(int)blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), out, g, row_bytes,
-                                                         h0 * d * esz, chunks, d);
+    summarize_kernel<false, MODE><<<(int)blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), out, g, row_bytes,
+                                                               h0 * d * esz, chunks, d);
   return cudaGetLastError();
+}
+
+cudaError_t launch_summarize(const void* x, float* out, const Geo& g, int heads_total, int h0, int hc, int d,
+                             spade_dtype dt, int mode, cudaStream_t s) {
+  if (mode == 1) return launch_summarize_m<1>(x, out, g, heads_total, h0, hc, d, dt, s);
+  if (mode == 2) return launch_summarize_m<2>(x, out, g, heads_total, h0, hc, d, dt, s);
+  return launch_summarize_m<0>(x, out, g, heads_total, h0, hc, d, dt, s);
 }
 
 }  // namespace spade

@@ -265,7 +265,22 @@ spade_status spade_summarize(const void* x, float* xmean, spade_geom g, int head
   if (!x || !xmean) return fail(SPADE_ERR_INVALID, "null pointer");
   if (!aligned16(x) || !aligned16(xmean)) return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
   if (heads < 1) return fail(SPADE_ERR_INVALID, "heads=%d", heads);
-  cudaError_t e = launch_summarize(x, xmean, make_geo(g), heads, 0, heads, d, dt, as_cuda(stream));
+  cudaError_t e = launch_summarize(x, xmean, make_geo(g), heads, 0, heads, d, dt, 0, as_cuda(stream));
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "summarize");
+}
+
+spade_status spade_summarize_mode(const void* x, float* out, spade_geom g, int heads, int d, spade_dtype dt,
+                                  spade_summary mode, spade_stream_t stream) {
+  if (mode != SPADE_SUM_MEAN && mode != SPADE_SUM_MAX && mode != SPADE_SUM_MIN)
+    return fail(SPADE_ERR_INVALID, "summary mode %d", (int)mode);
+  if (mode == SPADE_SUM_MEAN) return spade_summarize(x, out, g, heads, d, dt, stream);
+  spade_status st = check_geom(g);
+  if (st != SPADE_OK) return st;
+  if ((st = check_d_dt(d, dt)) != SPADE_OK) return st;
+  if (!x || !out) return fail(SPADE_ERR_INVALID, "null pointer");
+  if (!aligned16(x) || !aligned16(out)) return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  if (heads < 1) return fail(SPADE_ERR_INVALID, "heads=%d", heads);
+  cudaError_t e = launch_summarize(x, out, make_geo(g), heads, 0, heads, d, dt, (int)mode, as_cuda(stream));
   return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "summarize");
 }
 
@@ -436,6 +451,17 @@ spade_status spade_grouped_head_lists(const spade_geom* schemes, int n_schemes, 
 spade_status spade_grouped_attn(const void* q, const void* k, const void* v, void* out, const spade_geom* schemes,
                                 int n_schemes, const spade_head_scheme* table, int heads, int d, int text_tokens,
                                 spade_dtype dt, void* workspace, size_t ws_bytes, spade_stream_t stream) {
+  return spade_grouped_attn_ex(q, k, v, out, schemes, n_schemes, table, heads, d, text_tokens, dt, SPADE_SUM_MEAN,
+                               SPADE_SUM_MEAN, workspace, ws_bytes, stream);
+}
+
+spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, void* out, const spade_geom* schemes,
+                                   int n_schemes, const spade_head_scheme* table, int heads, int d, int text_tokens,
+                                   spade_dtype dt, spade_summary q_summary, spade_summary k_summary,
+                                   void* workspace, size_t ws_bytes, spade_stream_t stream) {
+  if ((q_summary != SPADE_SUM_MEAN && q_summary != SPADE_SUM_MAX && q_summary != SPADE_SUM_MIN) ||
+      (k_summary != SPADE_SUM_MEAN && k_summary != SPADE_SUM_MAX && k_summary != SPADE_SUM_MIN))
+    return fail(SPADE_ERR_INVALID, "summary modes %d/%d", (int)q_summary, (int)k_summary);
   GroupLayout L;
   spade_status st = plan_group(schemes, n_schemes, table, heads, d, text_tokens, L);
   if (st != SPADE_OK) return st;
@@ -459,8 +485,8 @@ spade_status spade_grouped_attn(const void* q, const void* k, const void* v, voi
       int j = i + 1;
       while (j < hs && hl[j] == hl[j - 1] + 1) ++j;
       const size_t o = (size_t)i * g.nb * d;
-      cudaError_t e = launch_summarize(q, qm + o, g, heads, hl[i], j - i, d, dt, s);
-      if (e == cudaSuccess) e = launch_summarize(k, km + o, g, heads, hl[i], j - i, d, dt, s);
+      cudaError_t e = launch_summarize(q, qm + o, g, heads, hl[i], j - i, d, dt, (int)q_summary, s);
+      if (e == cudaSuccess) e = launch_summarize(k, km + o, g, heads, hl[i], j - i, d, dt, (int)k_summary, s);
       if (e != cudaSuccess) return cuda_fail(e, "summarize");
       i = j;
     }

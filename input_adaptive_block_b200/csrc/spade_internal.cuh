@@ -80,7 +80,7 @@ __host__ __device__ inline int text_blocks(int text_tokens) { return (text_token
 cudaError_t launch_tile3d(const void* x, void* xt, const Geo& g, int heads, int d, spade_dtype dt,
                           cudaStream_t s);
 cudaError_t launch_summarize(const void* x, float* out, const Geo& g, int heads_total, int h0, int hc, int d,
-                             spade_dtype dt, cudaStream_t s);
+                             spade_dtype dt, int mode, cudaStream_t s);
 cudaError_t launch_estimate_tc(const float* qm, const float* km, float* prob, int heads, int nb, int d, int* status,
                                cudaStream_t s);
 cudaError_t launch_estimate(const float* qm, const float* km, float* prob, int heads, int nb, int d,
