@@ -49,7 +49,7 @@ import numpy as np
 
 __all__ = [
     "block_tokens", "valid_counts", "tile3d", "untile3d", "summarize", "estimate",
-    "select_row", "select", "selection_margin", "attention_rows", "block_sparse_attention",
+    "select_row", "select", "selection_margin", "window_blocks", "attention_rows", "block_sparse_attention",
     "dense_attention", "pipeline", "kept_token_pairs",
     "block_sics", "sics", "choose_schemes",
 ]
@@ -156,14 +156,34 @@ def estimate(qmean: np.ndarray, kmean: np.ndarray) -> np.ndarray:
 # 4. Index search: smallest diagonal-containing set reaching mass tau
 # ---------------------------------------------------------------------------
 
-def select_row(p: np.ndarray, i: int, tau: float) -> List[int]:
-    """Kept key blocks (ascending) for query block i of one head."""
+def window_blocks(geom: Sequence[int], i: int, radius: Sequence[int]) -> List[int]:
+    """Static window of query block i: the blocks whose (block-t, block-y,
+    block-x) coordinates lie within radius = (rt, ry, rx) of block i's
+    (technical summary, Methodology 2, Policy Application: "balancing static
+    windows and dynamic selection").  Radius (0, 0, 0) is block i alone."""
+    T, H, W, bt, bh, bw = (int(g) for g in geom)
+    nbt, nbh, nbw = -(-T // bt), -(-H // bh), -(-W // bw)
+    it, iy, ix = i // (nbh * nbw), (i // nbw) % nbh, i % nbw
+    out = []
+    for j in range(nbt * nbh * nbw):
+        jt, jy, jx = j // (nbh * nbw), (j // nbw) % nbh, j % nbw
+        if abs(jt - it) <= radius[0] and abs(jy - iy) <= radius[1] and abs(jx - ix) <= radius[2]:
+            out.append(j)
+    return out
+
+
+def select_row(p: np.ndarray, i: int, tau: float, window: Optional[Sequence[int]] = None) -> List[int]:
+    """Kept key blocks (ascending) for query block i of one head.  The
+    static window (default: block i alone -- the diagonal) is kept first and
+    its mass counts; the other blocks follow in descending probability."""
     nb = len(p)
     if tau >= 1.0:
         return list(range(nb))
-    kept = [i]
-    mass = float(p[i])
-    others = sorted((j for j in range(nb) if j != i), key=lambda j: (-p[j], j))
+    win = sorted(set(window)) if window is not None else [i]
+    kept = list(win)
+    mass = float(sum(float(p[j]) for j in win))
+    inwin = set(win)
+    others = sorted((j for j in range(nb) if j not in inwin), key=lambda j: (-p[j], j))
     for j in others:
         if mass >= tau:
             break
@@ -186,7 +206,7 @@ def select(P: np.ndarray, taus: Sequence[float]) -> Tuple[np.ndarray, np.ndarray
     return cnt, idx
 
 
-def selection_margin(p: np.ndarray, i: int, tau: float) -> float:
+def selection_margin(p: np.ndarray, i: int, tau: float, window: Optional[Sequence[int]] = None) -> float:
     """How far row i is from changing its kept set, in the estimator's score
     units (pooled logits; a probability ratio p_a/p_b is a score difference
     ln(p_a/p_b)).  It is the smallest of
@@ -200,12 +220,14 @@ def selection_margin(p: np.ndarray, i: int, tau: float) -> float:
     nb = len(p)
     if tau >= 1.0:
         return math.inf
-    others = sorted((j for j in range(nb) if j != i), key=lambda j: (-p[j], j))
+    win = sorted(set(window)) if window is not None else [i]
+    inwin = set(win)
+    others = sorted((j for j in range(nb) if j not in inwin), key=lambda j: (-p[j], j))
 
     def sens(c):
         return max(c * (1.0 - c), 1e-300)
 
-    mass = float(p[i])
+    mass = float(sum(float(p[j]) for j in win))
     k = 0
     prev = None
     while mass < tau and k < len(others):
@@ -214,7 +236,7 @@ def selection_margin(p: np.ndarray, i: int, tau: float) -> float:
         k += 1
     if mass < tau:            # every block kept because the mass never reached tau
         return 0.0
-    if k == 0:                # the diagonal alone reached tau
+    if k == 0:                # the diagonal (or the static window) alone reached tau
         return (mass - tau) / sens(mass)
     m = min((tau - prev) / sens(prev), (mass - tau) / sens(mass))
     if k < len(others):

@@ -363,3 +363,52 @@ def test_summarize_modes_agree_on_constant_blocks():
         x[toks] = vals[b]
     for m in ("mean", "max", "min"):
         assert np.allclose(O.summarize(x, geom, m)[0, :, 0], vals)
+
+
+# ---- static windows merged with dynamic selection ----
+
+def test_window_blocks_by_coordinates():
+    geom = (5, 9, 10, 2, 4, 4)                       # 3 x 3 x 3 blocks
+    assert O.window_blocks(geom, 13, (0, 0, 0)) == [13]
+    assert O.window_blocks(geom, 13, (1, 1, 1)) == list(range(27))   # the centre block's neighbourhood is all
+    assert O.window_blocks(geom, 0, (0, 0, 1)) == [0, 1]
+    assert O.window_blocks(geom, 0, (1, 0, 0)) == [0, 9]
+    assert O.window_blocks(geom, 26, (0, 1, 1)) == [22, 23, 25, 26]
+
+
+def test_select_with_radius_zero_window_is_the_diagonal_rule():
+    rng = np.random.default_rng(12)
+    geom = (4, 8, 8, 2, 4, 4)
+    for _ in range(20):
+        p = rng.dirichlet(np.full(8, 0.4))
+        i = int(rng.integers(0, 8))
+        tau = float(rng.uniform(0.3, 0.99))
+        assert O.select_row(p, i, tau, O.window_blocks(geom, i, (0, 0, 0))) == O.select_row(p, i, tau)
+
+
+def test_select_with_window_brute_force():
+    """The kept set is the smallest superset of the window whose mass reaches
+    tau, ties broken toward the larger mass then the lexicographically
+    smaller ids -- checked by enumerating every superset."""
+    import itertools
+    rng = np.random.default_rng(13)
+    geom = (4, 8, 8, 2, 4, 4)                        # 8 blocks
+    for _ in range(30):
+        p = rng.dirichlet(np.full(8, 0.5))
+        i = int(rng.integers(0, 8))
+        win = O.window_blocks(geom, i, (0, 1, 0))
+        tau = float(rng.uniform(0.3, 0.98))
+        got = O.select_row(p, i, tau, win)
+        rest = [j for j in range(8) if j not in win]
+        best = None
+        for r in range(len(rest) + 1):
+            for extra in itertools.combinations(rest, r):
+                s = sorted(win + list(extra))
+                m = float(p[s].sum())
+                if m >= tau or len(s) == 8:
+                    key = (len(s), -m, s)
+                    best = key if best is None or key < best else best
+            if best is not None:
+                break
+        assert got == best[2], (p, i, tau, got, best)
+        assert set(win) <= set(got)
