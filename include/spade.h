@@ -125,6 +125,19 @@ spade_status spade_estimate(const float* qmean, const float* kmean, float* prob,
 spade_status spade_select(const float* prob, const float* tau_host, int* cnt, int* idx,
                           int heads, int nb, spade_stream_t stream);
 
+/* Static windows merged with dynamic selection (Methodology 2, Policy
+ * Application: "balancing static windows and dynamic selection").  The
+ * window of query block i -- the blocks whose (block-t, block-y, block-x)
+ * coordinates in geometry g lie within radius_per_head[h] = (rt, ry, rx) of
+ * block i's -- takes the place of the diagonal: it is always kept and its
+ * mass counts first; the other blocks follow by descending probability
+ * until the mass reaches tau.  Radius (0, 0, 0) is exactly spade_select.
+ * prob: [heads, nb, nb] with nb = the block count of g; radius_per_head:
+ * host int32 [heads][3], non-negative.  Same outputs and limits as
+ * spade_select. */
+spade_status spade_select_window(const float* prob, const float* tau_per_head, const int* radius_per_head,
+                                 spade_geom g, int* cnt, int* idx, int heads, spade_stream_t stream);
+
 /* ---- step 5: flash block-sparse attention (one scheme) -------------------
  * Methodology 3, "Flash Block-Sparse Attention": exact softmax attention of
  * every valid query token of block i over the valid tokens of its kept key
@@ -187,13 +200,17 @@ spade_status spade_grouped_attn(const void* q, const void* k, const void* v, voi
                                 void* workspace, size_t ws_bytes, spade_stream_t stream);
 
 /* spade_grouped_attn with the Summarizer reduce chosen for Q and for K
- * (the estimator then scores the pooled Q and K summaries as usual);
- * spade_grouped_attn is this call with SPADE_SUM_MEAN for both. */
+ * (the estimator then scores the pooled Q and K summaries as usual) and an
+ * optional static window per head (window_radius: host int32 [heads][3]
+ * block radii (rt, ry, rx), see spade_select_window; NULL keeps the
+ * diagonal rule).  spade_grouped_attn is this call with SPADE_SUM_MEAN for
+ * both and no window. */
 spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, void* out,
                                    const spade_geom* schemes, int n_schemes,
                                    const spade_head_scheme* table, int heads, int d,
                                    int text_tokens, spade_dtype dt,
                                    spade_summary q_summary, spade_summary k_summary,
+                                   const int* window_radius,
                                    void* workspace, size_t ws_bytes, spade_stream_t stream);
 
 /* Where, inside a grouped workspace, head `head`'s kept lists live (byte

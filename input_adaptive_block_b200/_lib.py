@@ -46,7 +46,9 @@ SIGNATURES = {
     "spade_summarize_mode": (c_int, [c_void_p, c_void_p, SpadeGeom, c_int, c_int, c_int, c_int, c_void_p]),
     "spade_grouped_attn_ex": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SpadeGeom), c_int,
                                       POINTER(SpadeHeadScheme), c_int, c_int, c_int, c_int, c_int, c_int,
-                                      c_void_p, c_size_t, c_void_p]),
+                                      c_void_p, c_void_p, c_size_t, c_void_p]),
+    "spade_select_window": (c_int, [c_void_p, POINTER(c_float), POINTER(ctypes.c_int), SpadeGeom, c_void_p,
+                                    c_void_p, c_int, c_void_p]),
     "spade_sics_workspace_bytes": (c_size_t, [POINTER(SpadeGeom), c_int, c_int]),
     "spade_sics": (c_int, [c_void_p, c_void_p, POINTER(SpadeGeom), c_int, c_int, c_int, c_int, c_void_p, c_void_p,
                            c_void_p, c_size_t, c_void_p]),

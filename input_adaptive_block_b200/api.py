@@ -17,7 +17,7 @@ from ._lib import SpadeGeom, SpadeHeadScheme, check
 __all__ = [
     "geom", "dtype_code", "tile3d", "summarize", "estimate", "select", "attn_workspace_bytes",
     "block_sparse_attn", "block_sparse_attn_noalloc", "grouped_workspace_bytes", "grouped_attn", "grouped_head_lists",
-    "last_device_status", "selftest_bounded_wait", "num_blocks", "sics_workspace_bytes", "sics",
+    "last_device_status", "selftest_bounded_wait", "num_blocks", "sics_workspace_bytes", "sics", "select_window",
 ]
 
 
@@ -107,6 +107,23 @@ def select(prob: torch.Tensor, taus: Sequence[float], cnt: Optional[torch.Tensor
     return cnt, idx
 
 
+def select_window(prob: torch.Tensor, taus: Sequence[float], radius, g, cnt: Optional[torch.Tensor] = None,
+                  idx: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Selection with a static window per head: radius = (rt, ry, rx) for
+    every head, or one such triple per head."""
+    heads, nb, _ = prob.shape
+    if cnt is None:
+        cnt = torch.empty(heads, nb, dtype=torch.int32, device=prob.device)
+    if idx is None:
+        idx = torch.full((heads, nb, nb), -1, dtype=torch.int32, device=prob.device)
+    rad = list(radius) if len(radius) == heads and hasattr(radius[0], "__len__") else [tuple(radius)] * heads
+    rad_arr = (ctypes.c_int * (3 * heads))(*[int(r) for t in rad for r in t])
+    tau_arr = (ctypes.c_float * heads)(*[float(t) for t in taus])
+    check(_lib.load().spade_select_window(_dev(prob, "prob"), tau_arr, rad_arr, geom(g), _dev(cnt, "cnt"),
+                                          _dev(idx, "idx"), heads, _stream(stream)), "spade_select_window")
+    return cnt, idx
+
+
 def attn_workspace_bytes(g, heads: int, d: int, text_tokens: int = 0) -> int:
     return int(_lib.load().spade_attn_workspace_bytes(geom(g), heads, d, text_tokens))
 
@@ -162,9 +179,10 @@ def grouped_workspace_bytes(schemes, table, d: int, text_tokens: int = 0) -> int
 
 def grouped_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, schemes, table, text_tokens: int = 0,
                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                 stream=None, summary=("mean", "mean")) -> torch.Tensor:
+                 stream=None, summary=("mean", "mean"), window=None) -> torch.Tensor:
     """table: per head (scheme index, tau, dense); summary: the Q and K
-    Summarizer reduces ("mean", "max" or "min")."""
+    Summarizer reduces ("mean", "max" or "min"); window: optional static
+    window block radii (rt, ry, rx) per head."""
     heads, d = q.shape[1], q.shape[2]
     gs, rows = _tables(schemes, table)
     if out is None:
@@ -172,7 +190,7 @@ def grouped_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, schemes, tab
     if workspace is None:
         need = int(_lib.load().spade_grouped_workspace_bytes(gs, len(schemes), rows, heads, d, text_tokens))
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    if tuple(summary) == ("mean", "mean"):
+    if tuple(summary) == ("mean", "mean") and window is None:
         check(_lib.load().spade_grouped_attn(
             _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), gs, len(schemes), rows, heads, d,
             text_tokens, dtype_code(q.dtype), _dev(workspace, "workspace"), workspace.numel(), _stream(stream)),
@@ -181,6 +199,7 @@ def grouped_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, schemes, tab
         check(_lib.load().spade_grouped_attn_ex(
             _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), gs, len(schemes), rows, heads, d,
             text_tokens, dtype_code(q.dtype), SUMMARY[summary[0]], SUMMARY[summary[1]],
+            (ctypes.c_int * (3 * heads))(*[int(r) for t in window for r in t]) if window is not None else None,
             _dev(workspace, "workspace"), workspace.numel(), _stream(stream)), "spade_grouped_attn_ex")
     return out
 

@@ -20,11 +20,16 @@ namespace {
 
 struct SelectTaus {
   float tau[SPADE_SELECT_MAX_HEADS];
+  // static windows (WIN kernels only): block radii per head and the block grid
+  unsigned char rad[SPADE_SELECT_MAX_HEADS][3];
+  int nbh, nbw;
 };
 
 constexpr int kSelWarps = 8;
 
-template <int NPL>
+// WIN: the static window of block radii (rt, ry, rx) around i replaces the
+// diagonal: its blocks are kept first and their mass counts toward tau.
+template <int NPL, bool WIN>
 __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __restrict__ prob,
                                                                const __grid_constant__ SelectTaus taus,
                                                                int* __restrict__ cnt, int* __restrict__ idx,
@@ -50,14 +55,28 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __r
   }
   __syncwarp();
   const float tau = taus.tau[h];
-  const float diag = b[i];
   // lane owns j in [lane*NPL, lane*NPL + NPL): contiguous, so ascending output is a lane-order scan
   float v[NPL];
+  uint32_t win = 0;   // bit e: element lane*NPL+e lies in the window (always kept)
 #pragma unroll
   for (int e = 0; e < NPL; ++e) {
     const int j = lane * NPL + e;
-    v[e] = (j < nb && j != i) ? b[j] : -1.0f;   // -1: never reaches a non-negative threshold
+    bool in = j == i;
+    if (WIN && j < nb) {
+      const int it = i / (taus.nbh * taus.nbw), iy = (i / taus.nbw) % taus.nbh, ix = i % taus.nbw;
+      const int jt = j / (taus.nbh * taus.nbw), jy = (j / taus.nbw) % taus.nbh, jx = j % taus.nbw;
+      in = abs(jt - it) <= taus.rad[h][0] && abs(jy - iy) <= taus.rad[h][1] && abs(jx - ix) <= taus.rad[h][2];
+    }
+    if (in && j < nb) win |= 1u << e;
+    v[e] = (j < nb && !in) ? b[j] : -1.0f;   // -1: never reaches a non-negative threshold
   }
+  // mass of the window (just p_ii without one: adding zeros is exact)
+  float diag = 0.f;
+#pragma unroll
+  for (int e = 0; e < NPL; ++e)
+    if (win & (1u << e)) diag += b[lane * NPL + e];
+#pragma unroll
+  for (int o = 16; o; o >>= 1) diag += __shfl_xor_sync(0xffffffffu, diag, o);
   uint32_t keep = 0;   // bit e: element lane*NPL+e kept
   bool keep_all = tau >= 1.0f;
   if (!keep_all && diag < tau) {
@@ -113,8 +132,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __r
     for (int e = 0; e < NPL; ++e)
       if (lane * NPL + e < nb) keep |= 1u << e;
   } else {
-    const int di = i - lane * NPL;                 // the diagonal is always kept
-    if (di >= 0 && di < NPL) keep |= 1u << di;
+    keep |= win;                                   // the diagonal (or the static window) is always kept
   }
   const int mine = __popc(keep);
   int pre = mine;
@@ -211,26 +229,37 @@ __global__ void __launch_bounds__(kWlThreads) worklist_kernel(const __grid_const
 }
 
 template <int NPL>
-cudaError_t launch_select_t(const float* prob, const SelectTaus& t, int* cnt, int* idx, int heads, int nb,
+cudaError_t launch_select_t(const float* prob, const SelectTaus& t, bool win, int* cnt, int* idx, int heads, int nb,
                             cudaStream_t s) {
   const long long rows = (long long)heads * nb;
   const int blocks = (int)((rows + kSelWarps - 1) / kSelWarps);
-  select_kernel<NPL><<<blocks, kSelWarps * 32, 0, s>>>(prob, t, cnt, idx, heads, nb);
+  if (win) select_kernel<NPL, true><<<blocks, kSelWarps * 32, 0, s>>>(prob, t, cnt, idx, heads, nb);
+  else select_kernel<NPL, false><<<blocks, kSelWarps * 32, 0, s>>>(prob, t, cnt, idx, heads, nb);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_select(const float* prob, const float* tau_host, int* cnt, int* idx, int heads, int nb,
-                          cudaStream_t s) {
-  SelectTaus t;
+                          cudaStream_t s, const int* radius_host, const Geo* g) {
+  static SelectTaus t;   // host staging (large); launches copy it into the parameter buffer
   for (int h = 0; h < heads; ++h) t.tau[h] = tau_host[h];
+  bool win = false;
+  if (radius_host && g) {
+    for (int h = 0; h < heads; ++h)
+      for (int a = 0; a < 3; ++a) {
+        t.rad[h][a] = (unsigned char)(radius_host[3 * h + a] > 255 ? 255 : radius_host[3 * h + a]);
+        win = win || radius_host[3 * h + a] > 0;
+      }
+    t.nbh = g->nbh;
+    t.nbw = g->nbw;
+  }
   const int npl = (nb + 31) / 32;
-  if (npl <= 4) return launch_select_t<4>(prob, t, cnt, idx, heads, nb, s);
-  if (npl <= 8) return launch_select_t<8>(prob, t, cnt, idx, heads, nb, s);
-  if (npl <= 16) return launch_select_t<16>(prob, t, cnt, idx, heads, nb, s);
-  if (npl <= 24) return launch_select_t<24>(prob, t, cnt, idx, heads, nb, s);
-  return launch_select_t<32>(prob, t, cnt, idx, heads, nb, s);
+  if (npl <= 4) return launch_select_t<4>(prob, t, win, cnt, idx, heads, nb, s);
+  if (npl <= 8) return launch_select_t<8>(prob, t, win, cnt, idx, heads, nb, s);
+  if (npl <= 16) return launch_select_t<16>(prob, t, win, cnt, idx, heads, nb, s);
+  if (npl <= 24) return launch_select_t<24>(prob, t, win, cnt, idx, heads, nb, s);
+  return launch_select_t<32>(prob, t, win, cnt, idx, heads, nb, s);
 }
 
 cudaError_t launch_worklist(const AttnArgs& a, cudaStream_t s) {

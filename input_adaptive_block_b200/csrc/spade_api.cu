@@ -311,6 +311,23 @@ spade_status spade_select(const float* prob, const float* tau_host, int* cnt, in
   return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "select");
 }
 
+spade_status spade_select_window(const float* prob, const float* tau_host, const int* radius_host, spade_geom g,
+                                 int* cnt, int* idx, int heads, spade_stream_t stream) {
+  spade_status st = check_geom(g);
+  if (st != SPADE_OK) return st;
+  if (!prob || !tau_host || !radius_host || !cnt || !idx) return fail(SPADE_ERR_INVALID, "null pointer");
+  if (heads < 1 || heads > SPADE_SELECT_MAX_HEADS) return fail(SPADE_ERR_UNSUPPORTED, "heads=%d (1..1024)", heads);
+  const Geo gg = make_geo(g);
+  if (gg.nb > SPADE_SELECT_MAX_NB) return fail(SPADE_ERR_UNSUPPORTED, "nb=%d above %d", gg.nb, SPADE_SELECT_MAX_NB);
+  for (int h = 0; h < heads; ++h) {
+    if (!(tau_host[h] > 0.f && tau_host[h] <= 1e30f)) return fail(SPADE_ERR_INVALID, "tau[%d] must be > 0", h);
+    for (int a = 0; a < 3; ++a)
+      if (radius_host[3 * h + a] < 0) return fail(SPADE_ERR_INVALID, "window radius of head %d is negative", h);
+  }
+  cudaError_t e = launch_select(prob, tau_host, cnt, idx, heads, gg.nb, as_cuda(stream), radius_host, &gg);
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "select");
+}
+
 size_t spade_attn_workspace_bytes(spade_geom g, int heads, int d, int text_tokens) {
   (void)d;
   if (heads < 1 || text_tokens < 0 || g.bt <= 0 || g.bh <= 0 || g.bw <= 0 || g.T <= 0 || g.H <= 0 || g.W <= 0)
@@ -452,13 +469,18 @@ spade_status spade_grouped_attn(const void* q, const void* k, const void* v, voi
                                 int n_schemes, const spade_head_scheme* table, int heads, int d, int text_tokens,
                                 spade_dtype dt, void* workspace, size_t ws_bytes, spade_stream_t stream) {
   return spade_grouped_attn_ex(q, k, v, out, schemes, n_schemes, table, heads, d, text_tokens, dt, SPADE_SUM_MEAN,
-                               SPADE_SUM_MEAN, workspace, ws_bytes, stream);
+                               SPADE_SUM_MEAN, nullptr, workspace, ws_bytes, stream);
 }
 
 spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, void* out, const spade_geom* schemes,
                                    int n_schemes, const spade_head_scheme* table, int heads, int d, int text_tokens,
                                    spade_dtype dt, spade_summary q_summary, spade_summary k_summary,
-                                   void* workspace, size_t ws_bytes, spade_stream_t stream) {
+                                   const int* window_radius, void* workspace, size_t ws_bytes,
+                                   spade_stream_t stream) {
+  if (window_radius)
+    for (int h = 0; h < heads; ++h)
+      for (int a = 0; a < 3; ++a)
+        if (window_radius[3 * h + a] < 0) return fail(SPADE_ERR_INVALID, "window radius of head %d is negative", h);
   if ((q_summary != SPADE_SUM_MEAN && q_summary != SPADE_SUM_MAX && q_summary != SPADE_SUM_MIN) ||
       (k_summary != SPADE_SUM_MEAN && k_summary != SPADE_SUM_MAX && k_summary != SPADE_SUM_MIN))
     return fail(SPADE_ERR_INVALID, "summary modes %d/%d", (int)q_summary, (int)k_summary);
@@ -496,9 +518,15 @@ spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, 
     cudaError_t e = run_estimate(qm, km, prob, hs, g.nb, d, st, s);
     if (e != cudaSuccess) return cuda_fail(e, "estimate");
     std::vector<float> taus(hs);
-    for (int i = 0; i < hs; ++i) taus[i] = table[hl[i]].tau;
+    std::vector<int> rad(3 * hs, 0);
+    for (int i = 0; i < hs; ++i) {
+      taus[i] = table[hl[i]].tau;
+      if (window_radius)
+        for (int a = 0; a < 3; ++a) rad[3 * i + a] = window_radius[3 * hl[i] + a];
+    }
     e = launch_select(prob, taus.data(), reinterpret_cast<int*>(ws + L.cnt[sc]),
-                      reinterpret_cast<int*>(ws + L.idx[sc]), hs, g.nb, s);
+                      reinterpret_cast<int*>(ws + L.idx[sc]), hs, g.nb, s, window_radius ? rad.data() : nullptr,
+                      &g);
     if (e != cudaSuccess) return cuda_fail(e, "select");
   }
   // step 5: one grouped launch over every head

@@ -86,7 +86,7 @@ cudaError_t launch_estimate_tc(const float* qm, const float* km, float* prob, in
 cudaError_t launch_estimate(const float* qm, const float* km, float* prob, int heads, int nb, int d,
                             cudaStream_t s);
 cudaError_t launch_select(const float* prob, const float* tau_host, int* cnt, int* idx, int heads, int nb,
-                          cudaStream_t s);
+                          cudaStream_t s, const int* radius_host = nullptr, const Geo* g = nullptr);
 cudaError_t launch_worklist(const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 // Returns cudaErrorNotSupported if the shape is not for the tensor-core path.

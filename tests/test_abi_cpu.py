@@ -127,3 +127,16 @@ def test_sics_host_validation():
     other = (SpadeGeom * 2)(g1, SpadeGeom(21, 45, 81, 2, 8, 8))
     assert call(args(c=other, n=2)) == _lib.SPADE_ERR_INVALID
     assert b"different number of tokens" in lib.spade_last_error_message()
+
+
+def test_select_window_host_validation():
+    lib = _lib.load()
+    g = SpadeGeom(21, 45, 80, 2, 8, 8)
+    fake = ctypes.c_void_p(1 << 20)
+    taus = (ctypes.c_float * 1)(0.9)
+    rad = (ctypes.c_int * 3)(0, -1, 0)
+    assert lib.spade_select_window(fake, taus, rad, g, fake, fake, 1, None) == _lib.SPADE_ERR_INVALID
+    rad = (ctypes.c_int * 3)(0, 1, 0)
+    assert lib.spade_select_window(None, taus, rad, g, fake, fake, 1, None) == _lib.SPADE_ERR_INVALID
+    big = SpadeGeom(64, 64, 64, 2, 2, 2)            # 32768 blocks: above the selection limit
+    assert lib.spade_select_window(fake, taus, rad, big, fake, fake, 1, None) == _lib.SPADE_ERR_UNSUPPORTED
