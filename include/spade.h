@@ -246,6 +246,18 @@ spade_status spade_sics(const void* q, const void* k, const spade_geom* candidat
                         int heads, int d, spade_dtype dt, float* scores, int* choice,
                         void* workspace, size_t ws_bytes, spade_stream_t stream);
 
+/* ---- host <-> device head slices (pipelined execution from host memory) ----
+ * Copies the head slice [rows, h0 .. h0+hc, d] of a token-order array
+ * [rows, heads_total, d] between host memory (ideally pinned) and a
+ * contiguous device array [rows, hc, d]: to_device = 1 copies host -> device,
+ * 0 copies device -> host.  One strided 2-D copy on `stream`
+ * (asynchronous for pinned host memory); no kernels.  Lets a caller stream
+ * a layer through the GPU head group by head group -- heads are independent
+ * in every step -- overlapping the transfers of one group with the compute
+ * of another. */
+spade_status spade_copy_head_slice(void* device, void* host, int64_t rows, int heads_total, int h0, int hc,
+                                   int d, spade_dtype dt, int to_device, spade_stream_t stream);
+
 /* ---- status ---------------------------------------------------------------
  * spade_last_device_status synchronises `stream`, returns the latched device
  * status (SPADE_OK or SPADE_ERR_TIMEOUT) and clears it. */

@@ -49,6 +49,8 @@ SIGNATURES = {
                                       c_void_p, c_void_p, c_size_t, c_void_p]),
     "spade_select_window": (c_int, [c_void_p, POINTER(c_float), POINTER(ctypes.c_int), SpadeGeom, c_void_p,
                                     c_void_p, c_int, c_void_p]),
+    "spade_copy_head_slice": (c_int, [c_void_p, c_void_p, c_int64, c_int, c_int, c_int, c_int, c_int, c_int,
+                                      c_void_p]),
     "spade_sics_workspace_bytes": (c_size_t, [POINTER(SpadeGeom), c_int, c_int]),
     "spade_sics": (c_int, [c_void_p, c_void_p, POINTER(SpadeGeom), c_int, c_int, c_int, c_int, c_void_p, c_void_p,
                            c_void_p, c_size_t, c_void_p]),

@@ -18,6 +18,7 @@ __all__ = [
     "geom", "dtype_code", "tile3d", "summarize", "estimate", "select", "attn_workspace_bytes",
     "block_sparse_attn", "block_sparse_attn_noalloc", "grouped_workspace_bytes", "grouped_attn", "grouped_head_lists",
     "last_device_status", "selftest_bounded_wait", "num_blocks", "sics_workspace_bytes", "sics", "select_window",
+    "grouped_attn_from_host",
 ]
 
 
@@ -202,6 +203,71 @@ def grouped_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, schemes, tab
             (ctypes.c_int * (3 * heads))(*[int(r) for t in window for r in t]) if window is not None else None,
             _dev(workspace, "workspace"), workspace.numel(), _stream(stream)), "spade_grouped_attn_ex")
     return out
+
+
+def grouped_attn_from_host(qh: torch.Tensor, kh: torch.Tensor, vh: torch.Tensor, out_h: torch.Tensor, schemes,
+                           table, text_tokens: int = 0, head_chunk: int = 8, device=None,
+                           summary=("mean", "mean")) -> torch.Tensor:
+    """One layer from host memory to host memory, pipelined by head groups.
+
+    qh, kh, vh, out_h: host tensors [N (+text), heads, d] (pinned for the
+    copies to overlap).  Heads are independent in every step, so the layer
+    is streamed through the GPU in groups of head_chunk heads: the copy
+    stream brings group g in (strided 2-D copies, spade_copy_head_slice)
+    while the compute stream runs the grouped launch on group g-1 and the
+    copy stream returns finished groups.  Device buffers: two group slots.
+    Returns out_h after the call's work is enqueued; the caller synchronises
+    (or waits on the current stream, which this call joins at the end)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    rows, heads, d = qh.shape
+    dt = dtype_code(qh.dtype)
+    lib = _lib.load()
+    compute = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(dev)
+    groups = [(h0, min(head_chunk, heads - h0)) for h0 in range(0, heads, head_chunk)]
+    hcmax = max(hc for _, hc in groups)
+    # two slots x (q, k, v, out), each a flat buffer viewed as [rows, hc, d] for the group it holds
+    slots = [[torch.empty(rows * hcmax * d, dtype=qh.dtype, device=dev) for _ in range(4)] for _ in range(2)]
+    ws = [None, None]
+    loaded = [torch.cuda.Event() for _ in groups]
+    done = [torch.cuda.Event() for _ in groups]
+    returned = [torch.cuda.Event() for _ in groups]
+
+    def host_ptr(t):
+        return ctypes.c_void_p(t.data_ptr())
+
+    def load(gi):
+        h0, hc = groups[gi]
+        buf = slots[gi % 2]
+        if gi >= 2:
+            copy.wait_event(returned[gi - 2])             # the slot's previous group is back on the host
+        for src, dstb in zip((qh, kh, vh), buf[:3]):
+            check(lib.spade_copy_head_slice(dstb.data_ptr(), host_ptr(src), rows, heads, h0, hc, d, dt, 1,
+                                            copy.cuda_stream), "spade_copy_head_slice")
+        loaded[gi].record(copy)
+
+    with torch.cuda.stream(copy):
+        load(0)
+    for gi, (h0, hc) in enumerate(groups):
+        if gi + 1 < len(groups):
+            with torch.cuda.stream(copy):
+                load(gi + 1)
+        buf = slots[gi % 2]
+        compute.wait_event(loaded[gi])
+        q, k, v, o = (b[: rows * hc * d].view(rows, hc, d) for b in buf)
+        rows_t = list(table[h0: h0 + hc])
+        need = grouped_workspace_bytes(schemes, rows_t, d, text_tokens)
+        if ws[gi % 2] is None or ws[gi % 2].numel() < need:
+            ws[gi % 2] = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        out = grouped_attn(q, k, v, schemes, rows_t, text_tokens, out=o, workspace=ws[gi % 2], stream=compute,
+                           summary=summary)
+        done[gi].record(compute)
+        copy.wait_event(done[gi])
+        check(lib.spade_copy_head_slice(out.data_ptr(), host_ptr(out_h), rows, heads, h0, hc, d, dt, 0,
+                                        copy.cuda_stream), "spade_copy_head_slice")
+        returned[gi].record(copy)
+    compute.wait_stream(copy)
+    return out_h
 
 
 def grouped_head_lists(schemes, table, d: int, text_tokens: int, head: int) -> Tuple[int, int]:

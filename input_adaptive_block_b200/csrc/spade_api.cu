@@ -417,6 +417,23 @@ size_t spade_grouped_workspace_bytes(const spade_geom* schemes, int n_schemes, c
   return L.total;
 }
 
+spade_status spade_copy_head_slice(void* device, void* host, int64_t rows, int heads_total, int h0, int hc, int d,
+                                   spade_dtype dt, int to_device, spade_stream_t stream) {
+  if (!device || !host) return fail(SPADE_ERR_INVALID, "null pointer");
+  if (rows < 1 || heads_total < 1 || d < 1 || h0 < 0 || hc < 1 || h0 + hc > heads_total)
+    return fail(SPADE_ERR_INVALID, "slice [%d, %d) of %d heads, %lld rows", h0, h0 + hc, heads_total, (long long)rows);
+  if (dt != SPADE_F32 && dt != SPADE_BF16) return fail(SPADE_ERR_INVALID, "unknown dtype %d", (int)dt);
+  const size_t esz = dt == SPADE_BF16 ? 2 : 4;
+  const size_t hpitch = (size_t)heads_total * d * esz, dpitch = (size_t)hc * d * esz;
+  char* hp = static_cast<char*>(host) + (size_t)h0 * d * esz;
+  cudaError_t e = to_device
+                      ? cudaMemcpy2DAsync(device, dpitch, hp, hpitch, dpitch, (size_t)rows, cudaMemcpyHostToDevice,
+                                          as_cuda(stream))
+                      : cudaMemcpy2DAsync(hp, hpitch, device, dpitch, dpitch, (size_t)rows, cudaMemcpyDeviceToHost,
+                                          as_cuda(stream));
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "copy_head_slice");
+}
+
 size_t spade_sics_workspace_bytes(const spade_geom* candidates, int n_candidates, int heads) {
   if (!candidates || n_candidates < 1 || n_candidates > SPADE_MAX_SCHEMES || heads < 1) return 0;
   Geo g[SPADE_MAX_SCHEMES];

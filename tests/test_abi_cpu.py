@@ -140,3 +140,11 @@ def test_select_window_host_validation():
     assert lib.spade_select_window(None, taus, rad, g, fake, fake, 1, None) == _lib.SPADE_ERR_INVALID
     big = SpadeGeom(64, 64, 64, 2, 2, 2)            # 32768 blocks: above the selection limit
     assert lib.spade_select_window(fake, taus, rad, big, fake, fake, 1, None) == _lib.SPADE_ERR_UNSUPPORTED
+
+
+def test_copy_head_slice_host_validation():
+    lib = _lib.load()
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.spade_copy_head_slice(None, fake, 10, 4, 0, 2, 128, 1, 1, None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_copy_head_slice(fake, fake, 10, 4, 3, 2, 128, 1, 1, None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_copy_head_slice(fake, fake, 0, 4, 0, 2, 128, 1, 1, None) == _lib.SPADE_ERR_INVALID
