@@ -26,6 +26,7 @@ struct SelectTaus {
 };
 
 constexpr int kSelWarps = 8;
+constexpr int kFineBits = 18;   // low bits of theta bisected over the compacted candidates only
 
 // WIN: the static window of block radii (rt, ry, rx) around i replaces the
 // diagonal: its blocks are kept first and their mass counts toward tau.
@@ -81,7 +82,8 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __r
   bool keep_all = tau >= 1.0f;
   if (!keep_all && diag < tau) {
     uint32_t u = 0;
-    for (int bit = 29; bit >= 0; --bit) {           // p <= 1 < 2.0f = 0x40000000
+    // bits 29..18 over every element (p <= 1 < 2.0f = 0x40000000) ...
+    for (int bit = 29; bit >= kFineBits; --bit) {
       const uint32_t cand = u | (1u << bit);
       const float thr = __uint_as_float(cand);
       float s4[4] = {0.f, 0.f, 0.f, 0.f};                // four short chains instead of one long one
@@ -91,6 +93,49 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const float* __r
 #pragma unroll
       for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       if (diag + s >= tau) u = cand;
+    }
+    // ... then theta lies in [u, u + 2^kFineBits): the mass above that bracket
+    // counts as a constant and the remaining bits are bisected over the few
+    // elements inside it, compacted into the row buffer
+    {
+      const uint32_t top = u + (1u << kFineBits);
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      int mc = 0;
+#pragma unroll
+      for (int e = 0; e < NPL; ++e) {
+        const uint32_t bits = __float_as_uint(v[e]);
+        const bool pos = v[e] >= 0.f;
+        s4[e & 3] += (pos && bits >= top) ? v[e] : 0.f;
+        mc += (pos && bits >= u && bits < top);
+      }
+      float above = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+      int at = mc;                                   // inclusive scan of the candidate counts
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, at, o);
+        if (lane >= o) at += t;
+      }
+      const int ncand = __shfl_sync(0xffffffffu, at, 31);
+      at -= mc;
+      __syncwarp();                                  // every lane has read its row elements from b
+#pragma unroll
+      for (int e = 0; e < NPL; ++e) {
+        const uint32_t bits = __float_as_uint(v[e]);
+        if (v[e] >= 0.f && bits >= u && bits < top) b[at++] = v[e];
+      }
+      __syncwarp();
+      const float base = diag + above;
+      for (int bit = kFineBits - 1; bit >= 0; --bit) {
+        const uint32_t cand = u | (1u << bit);
+        const float thr = __uint_as_float(cand);
+        float s2 = 0.f;
+        for (int c = lane; c < ncand; c += 32) s2 += (b[c] >= thr) ? b[c] : 0.f;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        if (base + s2 >= tau) u = cand;
+      }
     }
     if (u == 0) {
       keep_all = true;                               // the mass never reaches tau
