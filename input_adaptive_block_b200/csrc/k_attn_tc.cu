@@ -10,14 +10,20 @@
 //  * 3D tiling by TMA: Q/K/V stay in token order [n, heads, d].  A 5-D tensor
 //    map {d, head, x, y, t} with box {64, 1, bw, bh, bt} lands one block of one
 //    head in shared memory as 128 rows x 128 B (slot order t, y, x), 128-byte
-//    swizzled -- the layout the MMA reads.  Out-of-grid slots are zero-filled
-//    by the TMA unit.  No tiled copy of Q/K/V is ever written.
+//    swizzled -- the layout the MMA reads.  Out-of-grid query slots are
+//    zero-filled by the TMA unit.  Key/value blocks clipped by the grid edge
+//    are loaded with a box of their own clipped extents (one map per edge
+//    case), so their valid tokens form a prefix of the tile: the score MMA's
+//    N, the P V MMA's K and the exponentials all stop at that prefix (rounded
+//    up to 16) instead of computing padded columns.  No tiled copy of Q/K/V is
+//    ever written.
 //  * tcgen05.mma (kind::f16, bf16 in, fp32 accumulate), issued by one thread.
-//    TMEM (512 columns): S0 | S1 (scores of key blocks j even / odd, fp32) |
-//    O (fp32) | P0 | P1 (bf16 probabilities).  S(j+2) is computed as soon as
-//    the softmax has read S(j) into registers (and is issued ahead of the
-//    other group's P V), so a score tile is normally waiting when the softmax
-//    reaches it; P V runs behind, reading P from TMEM.
+//    TMEM (512 columns): S0 | S1 | S2 (fp32 scores; key block g of the CTA
+//    uses buffer g % 3) | O (fp32).  The softmax reads S(g) into registers and
+//    writes P(g) (bf16) over the first half of the same buffer, where P V(g)
+//    reads it; S(g+3) is issued into the buffer once P V(g) has completed.
+//    With three buffers a group never waits for its previous P V before
+//    writing the next P, and two score tiles are normally computed ahead.
 //  * Warp specialisation: warp 0 hands out work and issues TMA loads (one K/V
 //    ring), warp 1 issues the Q K^T MMAs and warp 2 the P V MMAs (so neither
 //    stream's waits hold back the other's issue), warps 4-7 and 8-11 are two
@@ -49,8 +55,8 @@ namespace {
 constexpr int kAtomBytes = 128 * 128;        // 128 rows x 128 B: one 64-column swizzle atom of a tile
 constexpr int kMaxList = SPADE_TC_MAX_LIST;  // key blocks per work item staged in shared memory
 constexpr int kItemRing = 4;                 // work items in flight between the roles
-constexpr uint32_t kFullBlock = 1u << 31;    // extent code: every slot valid
-constexpr uint32_t kTextBlock = 1u << 30;    // extent code: text block (low bits = valid count)
+constexpr uint32_t kFullBlock = 1u << 31;    // extent code: every slot valid (low bits = 128)
+constexpr int kEdgeCases = 8;                // key/value maps per scheme: bit 0 t-, bit 1 y-, bit 2 x-edge
 
 // POLY_: when 1, every fourth column pair's exponential runs on the FMA pipe
 template <int D, int NS_, int POLY_>
@@ -65,13 +71,16 @@ struct Cfg {
   static constexpr int OFF_PLIST = OFF_KV + NS * TILE;            // producer's copy of the key list
   static constexpr int OFF_SEXT = OFF_PLIST + 4 * kMaxList;       // softmax: extent code per block
   static constexpr int OFF_DEC = OFF_SEXT + 4 * kMaxList;         // slot -> (t, y, x) per scheme
-  static constexpr int OFF_MREF = OFF_DEC + 4 * 128 * SPADE_MAX_SCHEMES;   // per-row reference max
+  static constexpr int OFF_NV = OFF_DEC + 4 * 128 * SPADE_MAX_SCHEMES;     // valid rows per K/V ring stage
+  static constexpr int OFF_MREF = OFF_NV + 4 * 16;                          // per-row reference max
   static constexpr int OFF_LX = OFF_MREF + 4 * 128;               // [2 groups][128 rows] row sums
   static constexpr int OFF_BAR = OFF_LX + 4 * 2 * 128;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;               // barriers + alignment slack
-  static constexpr uint32_t COL_S = 0;                            // S(j) at 128 (j % 2)
-  static constexpr uint32_t COL_O = 256;
-  static constexpr uint32_t COL_P = 256 + D;                      // P(j) at COL_P + 64 (j % 2)
+  // three score buffers: S(g) at 128 (g % 3), g counting the CTA's key
+  // blocks over all its items; P(g) (bf16 pairs) is written over the first 64
+  // columns of its own S buffer
+  static constexpr uint32_t COL_S = 0;
+  static constexpr uint32_t COL_O = 384;
   static constexpr uint32_t TMEM_COLS = 512;
   // warpgroup 0: producer, two MMA issuers, one idle warp; warpgroups 1-2:
   // softmax.  Registers per thread after the split (setmaxnreg): the split
@@ -84,8 +93,8 @@ struct Cfg {
 
 struct __align__(64) TcParams {
   CUtensorMap tm_q[SPADE_MAX_SCHEMES];
-  CUtensorMap tm_k[SPADE_MAX_SCHEMES];
-  CUtensorMap tm_v[SPADE_MAX_SCHEMES];
+  CUtensorMap tm_k[SPADE_MAX_SCHEMES][kEdgeCases];   // box = the clipped extents of each edge case
+  CUtensorMap tm_v[SPADE_MAX_SCHEMES][kEdgeCases];
   CUtensorMap tm_qt, tm_kt, tm_vt;          // text tokens (3-D maps), when present
   Geo geo[SPADE_MAX_SCHEMES];
   HeadInfo head[SPADE_MAX_HEADS];
@@ -196,6 +205,7 @@ __device__ __forceinline__ uint32_t pack_coord(const TcParams& p, const Item& I,
   return 0x80000000u | (uint32_t)(blk - I.nb);
 }
 
+// Query tile: the full box (out-of-grid slots zero-filled, slot order t, y, x).
 template <int D>
 __device__ __forceinline__ void load_tile(const TcParams& p, const CUtensorMap* vid, const CUtensorMap* txt,
                                           const Item& I, uint32_t pc, uint8_t* dst, uint64_t* bar) {
@@ -212,36 +222,58 @@ __device__ __forceinline__ void load_tile(const TcParams& p, const CUtensorMap* 
   }
 }
 
-// Extent code of key block `blk`: clipped (t, y, x) extents of a video block,
-// or the valid count of a text block, plus a flag when every slot is valid.
+// Edge case of a video block (bit 0: clipped in t, 1: in y, 2: in x) and its
+// number of valid tokens.
+__device__ __forceinline__ int edge_case(const Geo& g, int bi, int bj, int bk, int& nv) {
+  const int et = min(g.bt, g.T - bi * g.bt), eh = min(g.bh, g.H - bj * g.bh), ew = min(g.bw, g.W - bk * g.bw);
+  nv = et * eh * ew;
+  return (et < g.bt ? 1 : 0) | (eh < g.bh ? 2 : 0) | (ew < g.bw ? 4 : 0);
+}
+
+// Key or value tile into one ring stage: a video block through the map of its
+// edge case (valid tokens = the first nv rows, in t, y, x order), a text
+// block through the 3-D map (rows past the text end zero-filled).  The
+// stage's valid row count goes to *nv_slot before the barrier is armed with
+// the box's bytes (the arrival releases it to the MMA warps).  Whole warp,
+// uniform control flow.
+template <int D>
+__device__ __forceinline__ void load_kv_tile(const TcParams& p, const CUtensorMap (&vid)[kEdgeCases],
+                                             const CUtensorMap* txt, const Item& I, uint32_t pc, uint8_t* dst,
+                                             uint64_t* bar, volatile int* nv_slot) {
+  if (!(pc & 0x80000000u)) {
+    const Geo& g = p.geo[I.scheme];
+    const int bk = (int)(pc & 0xfffu), bj = (int)((pc >> 12) & 0x3ffu), bi = (int)(pc >> 22);
+    int nv;
+    const CUtensorMap* m = &vid[edge_case(g, bi, bj, bk, nv)];
+    *nv_slot = nv;
+    __syncwarp();
+    ptx::mbar_arrive_expect_tx_elect(bar, (uint32_t)(nv * 2 * D));
+#pragma unroll
+    for (int a = 0; a < D / 64; ++a)
+      ptx::tma_load_5d_elect(dst + a * kAtomBytes, m, bar, 64 * a, I.h, bk * g.bw, bj * g.bh, bi * g.bt);
+    return;
+  }
+  const int tb = (int)(pc & 0x7fffffffu);
+  *nv_slot = min(128, p.text_tokens - tb * 128);
+  __syncwarp();
+  ptx::mbar_arrive_expect_tx_elect(bar, (uint32_t)(128 * 2 * D));
+#pragma unroll
+  for (int a = 0; a < D / 64; ++a) ptx::tma_load_3d_elect(dst + a * kAtomBytes, txt, bar, 64 * a, I.h, tb * 128);
+}
+
+// Valid key columns of key block `blk` (a prefix of the tile: see
+// load_kv_tile), with a flag when all 128 are valid.
 __device__ __forceinline__ uint32_t extent_code(const TcParams& p, const Item& I, int blk) {
+  int valid;
   if (blk < I.nb) {
     const Geo& g = p.geo[I.scheme];
     int t0, y0, x0, et, eh, ew;
     block_box(g, blk, t0, y0, x0, et, eh, ew);
-    const bool full = et == g.bt && eh == g.bh && ew == g.bw;
-    return (uint32_t)et | ((uint32_t)eh << 8) | ((uint32_t)ew << 16) | (full ? kFullBlock : 0u);
+    valid = et * eh * ew;
+  } else {
+    valid = min(128, p.text_tokens - (blk - I.nb) * 128);
   }
-  const int valid = min(128, p.text_tokens - (blk - I.nb) * 128);
-  return (uint32_t)valid | kTextBlock | (valid >= 128 ? kFullBlock : 0u);
-}
-
-// Validity of the 128 key columns of a partial block as four 32-bit words
-// (warp-cooperative: lane l decides columns l, l+32, l+64, l+96; `dec` maps a
-// slot to its (t, y, x) offsets inside the box).
-__device__ __forceinline__ void key_mask(uint32_t code, const uint32_t* dec, int lane, uint32_t (&m)[4]) {
-  if (code & kTextBlock) {
-    const int valid = (int)(code & 0xffu);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) m[w] = __ballot_sync(0xffffffffu, lane + 32 * w < valid);
-    return;
-  }
-  const uint32_t et = code & 0xffu, eh = (code >> 8) & 0xffu, ew = (code >> 16) & 0xffu;
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    const uint32_t e = dec[lane + 32 * w];
-    m[w] = __ballot_sync(0xffffffffu, (e & 0xffu) < et && ((e >> 8) & 0xffu) < eh && (e >> 16) < ew);
-  }
+  return (uint32_t)valid | (valid >= 128 ? kFullBlock : 0u);
 }
 
 // ------------------------------------------------------- exp2 on the FMA pipe --
@@ -282,6 +314,7 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
   int* plist = reinterpret_cast<int*>(smem + C::OFF_PLIST);   // packed tile coordinates
   uint32_t* sext = reinterpret_cast<uint32_t*>(smem + C::OFF_SEXT);
   uint32_t* sdec = reinterpret_cast<uint32_t*>(smem + C::OFF_DEC);
+  volatile int* stage_nv = reinterpret_cast<volatile int*>(smem + C::OFF_NV);   // valid rows of each ring stage
   float* mref = reinterpret_cast<float*>(smem + C::OFF_MREF);  // [128 rows] reference max (log2 domain)
   float* lx = reinterpret_cast<float*>(smem + C::OFF_LX);      // [2 groups][128 rows] final row sums
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -289,23 +322,28 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
   uint64_t* kv_empty = bars + NS;
   uint64_t* q_full = bars + 2 * NS;
   uint64_t* q_empty = q_full + 1;
-  uint64_t* s_full = q_full + 2;      // [2] S(j) in TMEM (MMA commit)
-  uint64_t* s_free = q_full + 4;      // [2] S(j) read by its group (128 threads)
-  uint64_t* p_full = q_full + 6;      // [2] P(j) in TMEM (128 threads)
-  uint64_t* pv_done = q_full + 8;     // [2] P V(j) complete (MMA commit)
-  uint64_t* md = q_full + 10;         // [2] reference max of block j final (128 threads of its group)
-  uint64_t* o_full = q_full + 12;     // last P V of the item complete
-  uint64_t* o_free = q_full + 13;     // epilogue has read O (256 threads)
-  uint64_t* lx_bar = q_full + 14;     // both groups' final row sums published (256 threads)
-  uint64_t* stage_bar = q_full + 15;  // extent codes of the item staged (256 threads)
-  uint64_t* mma_fin = q_full + 16;    // [2] per MMA warp: all its MMAs complete
-  uint64_t* item_full = q_full + 18;
+  uint64_t* s_full = q_full + 2;      // [3] S(g) in TMEM buffer g % 3 (MMA commit)
+  uint64_t* p_full = q_full + 5;      // [3] P(g) written over S(g) (128 threads)
+  uint64_t* buf_free = q_full + 8;    // [3] P V(g) complete: buffer g % 3 may take S(g+3) (MMA commit)
+  uint64_t* md = q_full + 11;         // [2] reference max of block j final (128 threads of its group)
+  uint64_t* o_full = q_full + 13;     // last P V of the item complete
+  uint64_t* o_free = q_full + 14;     // epilogue has read O (256 threads)
+  uint64_t* lx_bar = q_full + 15;     // both groups' final row sums published (256 threads)
+  uint64_t* stage_bar = q_full + 16;  // extent codes of the item staged (256 threads)
+  uint64_t* mma_fin = q_full + 17;    // [2] per MMA warp: all its MMAs complete
+  uint64_t* item_full = q_full + 19;
   uint64_t* item_empty = item_full + kItemRing;
   int* item_ring = reinterpret_cast<int*>(item_empty + kItemRing);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_ring + kItemRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // A short key/value tile leaves the rows past its (16-rounded) prefix as
+  // the ring stage last held them; zeroing the ring once keeps them finite
+  // (0 * p = 0 in P V) before any tile has landed.
+  for (int e = threadIdx.x; e < NS * C::TILE / 16; e += blockDim.x)
+    reinterpret_cast<uint4*>(sKV)[e] = make_uint4(0u, 0u, 0u, 0u);
+  ptx::fence_proxy_async_smem();
   for (int e = threadIdx.x; e < p.n_schemes * 128; e += blockDim.x) {
     const Geo& g = p.geo[e >> 7];
     const int c = e & 127;
@@ -318,13 +356,13 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
     }
     ptx::mbar_init(q_full, 1);
     ptx::mbar_init(q_empty, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       ptx::mbar_init(&s_full[b], 1);
-      ptx::mbar_init(&s_free[b], 128);
       ptx::mbar_init(&p_full[b], 128);
-      ptx::mbar_init(&pv_done[b], 1);
-      ptx::mbar_init(&md[b], 128);
+      ptx::mbar_init(&buf_free[b], 1);
     }
+    ptx::mbar_init(&md[0], 128);
+    ptx::mbar_init(&md[1], 128);
     ptx::mbar_init(o_full, 1);
     ptx::mbar_init(o_free, 256);
     ptx::mbar_init(lx_bar, 256);
@@ -341,8 +379,10 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < p.n_schemes; ++s) {
       ptx::prefetch_tmap(&p.tm_q[s]);
-      ptx::prefetch_tmap(&p.tm_k[s]);
-      ptx::prefetch_tmap(&p.tm_v[s]);
+      for (int c = 0; c < kEdgeCases; ++c) {
+        ptx::prefetch_tmap(&p.tm_k[s][c]);
+        ptx::prefetch_tmap(&p.tm_v[s][c]);
+      }
     }
   }
   if (warp == 1) {
@@ -395,21 +435,20 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
       ptx::mbar_arrive_expect_tx_elect(q_full, C::TILE);
       load_tile<D>(p, &p.tm_q[I.scheme], &p.tm_qt, I, pack_coord(p, I, I.qb), sQ, q_full);
       qlast = li & 1;
-      auto push = [&](const CUtensorMap* vid, const CUtensorMap* txt, int pcw) -> bool {
+      auto push = [&](const CUtensorMap (&vid)[kEdgeCases], const CUtensorMap* txt, int pcw) -> bool {
         const int st = kvpos % NS;
         const uint32_t par = (kvpos / NS) & 1;
         if (!__all_sync(0xffffffffu, wait_bar(&kv_empty[st], par ^ 1, W))) return false;
-        ptx::mbar_arrive_expect_tx_elect(&kv_full[st], C::TILE);
-        load_tile<D>(p, vid, txt, I, (uint32_t)pcw, sKV + st * C::TILE, &kv_full[st]);
+        load_kv_tile<D>(p, vid, txt, I, (uint32_t)pcw, sKV + st * C::TILE, &kv_full[st], &stage_nv[st]);
         last_par[st] = par;
         used |= 1u << st;
         ++kvpos;
         return true;
       };
-      for (int j = 0; ok && j < 3 && j < I.n; ++j) ok = push(&p.tm_k[I.scheme], &p.tm_kt, plist[j]);
+      for (int j = 0; ok && j < 3 && j < I.n; ++j) ok = push(p.tm_k[I.scheme], &p.tm_kt, plist[j]);
       for (int j = 0; ok && j < I.n; ++j) {
-        if (j + 3 < I.n) ok = push(&p.tm_k[I.scheme], &p.tm_kt, plist[j + 3]);
-        if (ok) ok = push(&p.tm_v[I.scheme], &p.tm_vt, plist[j]);
+        if (j + 3 < I.n) ok = push(p.tm_k[I.scheme], &p.tm_kt, plist[j + 3]);
+        if (ok) ok = push(p.tm_v[I.scheme], &p.tm_vt, plist[j]);
       }
       __syncwarp();
       if (!ok) break;
@@ -434,11 +473,9 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
     // k < 3, at B + m + 2 (k - 3) otherwise; V_j at B + m + min(j + 1, n - 3) + j,
     // where m = min(n, 3) -- the producer's order K0, K1, K2, then K_{j+3}, V_j.
     const bool is_s = warp == 1;
-    constexpr uint32_t idesc_qk = make_idesc(128, 128, false);
     constexpr uint32_t idesc_pv = make_idesc(128, D, true);
     uint32_t base = 0;         // ring position of the item's first tile
-    uint32_t su[2] = {0, 0};   // S writes per buffer so far (S warp)
-    uint32_t pu[2] = {0, 0};   // P V reads per buffer so far (P V warp)
+    uint32_t g = 0;            // key blocks of this warp's stream so far (all items): buffer g % 3
     bool ok = true;
     for (int li = 0; ok; ++li) {
       const int slot = li % kItemRing;
@@ -456,16 +493,19 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint64_t qdesc = kmajor_desc(ptx::smem_u32(sQ));
-        for (int k = 0; ok && k < n; ++k) {
-          const int b = k & 1;
+        for (int k = 0; ok && k < n; ++k, ++g) {
+          const uint32_t b = g % 3;
           const uint32_t pos = base + (uint32_t)(k < 3 ? k : m + 2 * (k - 3));
           const int st = (int)(pos % NS);
           bool w = wait_bar(&kv_full[st], (pos / NS) & 1, W);
-          if (su[b] > 0) w = w && wait_bar(&s_free[b], (su[b] - 1) & 1, W);
+          // buffer b last held S(g-3) / P(g-3): wait until P V(g-3) has read it
+          if (g >= 3) w = w && wait_bar(&buf_free[b], (g / 3 - 1) & 1, W);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint64_t kdesc = kmajor_desc(ptx::smem_u32(sKV + st * C::TILE));
           const uint32_t ts = tmem + C::COL_S + 128 * b;
+          // N = valid key rows rounded up to 16 (the columns past it are masked by the softmax)
+          const uint32_t idesc_qk = make_idesc(128, (stage_nv[st] + 15) & ~15, false);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = (uint64_t)(((kk >> 2) * kAtomBytes + (kk & 3) * 32) >> 4);
@@ -473,29 +513,28 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
           }
           ptx::tc_commit_elect(&s_full[b]);
           ptx::tc_commit_elect(&kv_empty[st]);
-          ++su[b];
           if (k == n - 1) ptx::tc_commit_elect(q_empty);
         }
       } else {
-        for (int j = 0; ok && j < n; ++j) {
-          const int b = j & 1;
+        for (int j = 0; ok && j < n; ++j, ++g) {
+          const uint32_t b = g % 3;
           const uint32_t pos = base + (uint32_t)(m + (j + 1 < nk3 ? j + 1 : nk3) + j);
           const int st = (int)(pos % NS);
-          bool w = wait_bar(&p_full[b], pu[b] & 1, W);
+          bool w = wait_bar(&p_full[b], (g / 3) & 1, W);
           w = w && wait_bar(&kv_full[st], (pos / NS) & 1, W);
           if (j == 0) w = w && wait_bar(o_free, (li & 1) ^ 1, W);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint64_t vdesc = mnmajor_desc(ptx::smem_u32(sKV + st * C::TILE));
-          const uint32_t tp = tmem + C::COL_P + 64 * b;
+          const uint32_t tp = tmem + C::COL_S + 128 * b;   // P(g) over S(g)
           const uint32_t acc0 = j > 0 ? 1u : 0u;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
+          const int nk = (stage_nv[st] + 15) >> 4;       // K steps of 16 keys over the valid prefix
+#pragma unroll 1
+          for (int kk = 0; kk < nk; ++kk)
             ptx::mma_ts_elect(tmem + C::COL_O, tp + kk * 8, vdesc + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
                               kk > 0 ? 1u : acc0);
-          ptx::tc_commit_elect(&pv_done[b]);
+          ptx::tc_commit_elect(&buf_free[b]);
           ptx::tc_commit_elect(&kv_empty[st]);
-          ++pu[b];
           if (j == n - 1) ptx::tc_commit_elect(o_full);
         }
       }
@@ -515,12 +554,11 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
     const int row = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const int gtid = threadIdx.x - 128;                // 0..255 over both groups
-    const uint32_t tS = tmem + lane_base + C::COL_S + 128 * w;
-    const uint32_t tP = tmem + lane_base + C::COL_P + 64 * w;
     const uint32_t tO = tmem + lane_base + C::COL_O;
     const float sl2 = p.scale_log2;
     const float2 sl2x2 = make_float2(sl2, sl2);
     uint32_t nb_done[2] = {0, 0};                      // blocks of each group before this item
+    uint32_t g0 = 0;                                   // key blocks of all previous items
     bool ok = true;
     for (int li = 0; ok; ++li) {
       const int slot = li % kItemRing;
@@ -537,25 +575,22 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
       ptx::mbar_arrive(stage_bar);
       ok = wait_bar(stage_bar, li & 1, W);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      const uint32_t* dec = sdec + 128 * I.scheme;
       float l = 0.f;          // this group's share of the row sum, relative to m_seen
       float m_seen = 0.f;     // reference max at this group's last block
       for (int j = w; j < n; j += 2) {
-        const uint32_t kself = nb_done[w] + (uint32_t)(j >> 1);        // this group's block counter
-        ok = wait_bar(&s_full[w], kself & 1, W);
+        const uint32_t g = g0 + (uint32_t)j;           // the CTA's key-block counter: buffer g % 3
+        const uint32_t b = g % 3;
+        const uint32_t tS = tmem + lane_base + C::COL_S + 128 * b;
+        ok = wait_bar(&s_full[b], (g / 3) & 1, W);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         ptx::tc_fence_after();
         uint32_t sr[128];
-        ptx::tmem_ld128(tS, sr);
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&s_free[w]);                  // S buffer may take S(j+2)
-        const uint32_t code = sext[j];
-        if (!(code & kFullBlock)) {
-          uint32_t mw[4];
-          key_mask(code, dec, lane, mw);
+        ptx::tmem_ld128(tS, sr);                       // waits for the loads: P may now overwrite S
+        const int nv = (int)(sext[j] & 0xffu);         // valid key columns: a prefix
+        if (nv < 128) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (!((mw[c >> 5] >> (c & 31)) & 1u)) sr[c] = 0xff800000u;   // -inf
+            if (c >= nv) sr[c] = 0xff800000u;            // -inf
         }
         float mk[8];
 #pragma unroll
@@ -587,20 +622,17 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
         ptx::mbar_arrive(&md[w]);
         if (l != 0.f && m_seen != m_use) l *= ptx::ex2(m_seen - m_use);
         m_seen = m_use;
-        // P buffer w was last read by this group's previous block's P V
-        if (kself > 0) {
-          ok = wait_bar(&pv_done[w], (kself - 1) & 1, W);
-          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        }
-        // p = 2^(s*scale*log2e - m) in four 32-column chunks: FFMA2, exp2
-        // (SFU; with POLY, every fourth pair on the FMA pipe), row-sum FADD2,
-        // bf16 pack, TMEM store; masked columns are -inf and give 0
+        // p = 2^(s*scale*log2e - m) in 32-column chunks up to the valid
+        // prefix: FFMA2, exp2 (SFU; with POLY, every fourth pair on the FMA
+        // pipe), row-sum FADD2, bf16 pack, TMEM store; masked columns are
+        // -inf and give 0; chunks past the prefix are not read by P V
         {
           const float2 nm2 = make_float2(-m_use, -m_use);
           float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                             make_float2(0.f, 0.f)};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
+            if (32 * q >= nv) break;
             float2 pe[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c)
@@ -620,7 +652,7 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
             uint32_t pk[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c) pk[c] = ptx::pack_bf16x2(pe[c].x, pe[c].y);
-            ptx::tmem_st16_nowait(tP + 16 * q, pk);
+            ptx::tmem_st16_nowait(tS + 16 * q, pk);
           }
           const float2 a = __fadd2_rn(__fadd2_rn(acc4[0], acc4[1]), __fadd2_rn(acc4[2], acc4[3]));
           l += a.x + a.y;
@@ -629,8 +661,7 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
         if (__any_sync(0xffffffffu, raise)) {
           // O holds blocks < j relative to the old reference: rescale it once
           // P V(j-1) has landed (P V(j) waits for this group's P below)
-          const uint32_t kother = nb_done[w ^ 1] + (uint32_t)((j - 1) >> 1);
-          ok = wait_bar(&pv_done[w ^ 1], kother & 1, W);
+          ok = wait_bar(&buf_free[(g - 1) % 3], ((g - 1) / 3) & 1, W);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           ptx::tc_fence_after();
 #pragma unroll 1
@@ -643,7 +674,7 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
           }
         }
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&p_full[w]);
+        ptx::mbar_arrive(&p_full[b]);
       }
       if (!ok) break;
       // ---- epilogue: combine the groups' row sums, O / l -> bf16 -> token order
@@ -666,6 +697,7 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
       }
       nb_done[0] += (uint32_t)((n + 1) >> 1);
       nb_done[1] += (uint32_t)(n >> 1);
+      g0 += (uint32_t)n;
       const float inv = 1.0f / (lx[row] + lx[128 + row]);
       const Item E = get_item(p, it);   // re-read: nothing of the item stays live across the block loop
       long long tok = -1;
@@ -724,12 +756,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-bool map_video(CUtensorMap* m, const void* base, const Geo& g, int heads, int d) {
+// box = (et, eh, ew) tokens of one head: the block shape, or the clipped
+// extents of an edge block
+bool map_video(CUtensorMap* m, const void* base, const Geo& g, int heads, int d, int et, int eh, int ew) {
   const cuuint64_t es = 2;
   cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T};
   cuuint64_t strides[4] = {d * es, (cuuint64_t)heads * d * es, (cuuint64_t)g.W * heads * d * es,
                            (cuuint64_t)g.H * g.W * heads * d * es};
-  cuuint32_t box[5] = {64, 1, (cuuint32_t)g.bw, (cuuint32_t)g.bh, (cuuint32_t)g.bt};
+  cuuint32_t box[5] = {64, 1, (cuuint32_t)ew, (cuuint32_t)eh, (cuuint32_t)et};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -786,8 +820,15 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s, const char** why) 
   const int es = 2;
   for (int sc = 0; sc < a.n_schemes; ++sc) {
     const Geo& g = a.geo[sc];
-    if (!map_video(&tp.tm_q[sc], a.q, g, a.heads, a.d) || !map_video(&tp.tm_k[sc], a.k, g, a.heads, a.d) ||
-        !map_video(&tp.tm_v[sc], a.v, g, a.heads, a.d)) {
+    bool ok = map_video(&tp.tm_q[sc], a.q, g, a.heads, a.d, g.bt, g.bh, g.bw);
+    // key/value maps per edge case (cases the grid does not have repeat the full box)
+    const int lt = g.T - (g.nbt - 1) * g.bt, lh = g.H - (g.nbh - 1) * g.bh, lw = g.W - (g.nbw - 1) * g.bw;
+    for (int c = 0; ok && c < kEdgeCases; ++c) {
+      const int et = (c & 1) ? lt : g.bt, eh = (c & 2) ? lh : g.bh, ew = (c & 4) ? lw : g.bw;
+      ok = map_video(&tp.tm_k[sc][c], a.k, g, a.heads, a.d, et, eh, ew) &&
+           map_video(&tp.tm_v[sc][c], a.v, g, a.heads, a.d, et, eh, ew);
+    }
+    if (!ok) {
       *why = "tensor map encoding failed (video)";
       return cudaErrorInvalidValue;
     }
