@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
     // item's key list in shared memory; one elected lane takes the ticket,
     // publishes the item (or -1 at the end) to the other roles, and issues
     // each expect-tx / TMA load (elect.sync-predicated, no divergent branch).
-    // Ring order = MMA consumption order: K0, K1, K2, then K_{j+3}, V_j.
+    // Ring order = MMA consumption order: K0, K1, K2, then V_j, K_{j+3} (S(j+3) waits for P V(j) anyway).
     uint32_t kvpos = 0;
     uint32_t last_par[NS];
     uint32_t used = 0;
@@ -447,8 +447,8 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
       };
       for (int j = 0; ok && j < 3 && j < I.n; ++j) ok = push(p.tm_k[I.scheme], &p.tm_kt, plist[j]);
       for (int j = 0; ok && j < I.n; ++j) {
-        if (j + 3 < I.n) ok = push(p.tm_k[I.scheme], &p.tm_kt, plist[j + 3]);
-        if (ok) ok = push(p.tm_v[I.scheme], &p.tm_vt, plist[j]);
+        ok = push(p.tm_v[I.scheme], &p.tm_vt, plist[j]);
+        if (ok && j + 3 < I.n) ok = push(p.tm_k[I.scheme], &p.tm_kt, plist[j + 3]);
       }
       __syncwarp();
       if (!ok) break;
@@ -470,8 +470,8 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
     // control flow; one elected lane issues each tcgen05.mma / commit.
     //
     // Ring positions inside an item with n blocks (base B): K_k at B + k for
-    // k < 3, at B + m + 2 (k - 3) otherwise; V_j at B + m + min(j + 1, n - 3) + j,
-    // where m = min(n, 3) -- the producer's order K0, K1, K2, then K_{j+3}, V_j.
+    // k < 3, at B + m + 2 (k - 3) + 1 otherwise; V_j at B + m + j + min(j, n - 3),
+    // where m = min(n, 3) -- the producer's order K0, K1, K2, then V_j, K_{j+3}.
     const bool is_s = warp == 1;
     constexpr uint32_t idesc_pv = make_idesc(128, D, true);
     uint32_t base = 0;         // ring position of the item's first tile
@@ -495,7 +495,7 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
         const uint64_t qdesc = kmajor_desc(ptx::smem_u32(sQ));
         for (int k = 0; ok && k < n; ++k, ++g) {
           const uint32_t b = g % 3;
-          const uint32_t pos = base + (uint32_t)(k < 3 ? k : m + 2 * (k - 3));
+          const uint32_t pos = base + (uint32_t)(k < 3 ? k : m + 2 * (k - 3) + 1);
           const int st = (int)(pos % NS);
           bool w = wait_bar(&kv_full[st], (pos / NS) & 1, W);
           // buffer b last held S(g-3) / P(g-3): wait until P V(g-3) has read it
@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
       } else {
         for (int j = 0; ok && j < n; ++j, ++g) {
           const uint32_t b = g % 3;
-          const uint32_t pos = base + (uint32_t)(m + (j + 1 < nk3 ? j + 1 : nk3) + j);
+          const uint32_t pos = base + (uint32_t)(m + j + (j < nk3 ? j : nk3));
           const int st = (int)(pos % NS);
           bool w = wait_bar(&p_full[b], (g / 3) & 1, W);
           w = w && wait_bar(&kv_full[st], (pos / NS) & 1, W);
@@ -622,17 +622,17 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
         ptx::mbar_arrive(&md[w]);
         if (l != 0.f && m_seen != m_use) l *= ptx::ex2(m_seen - m_use);
         m_seen = m_use;
-        // p = 2^(s*scale*log2e - m) in 32-column chunks up to the valid
-        // prefix: FFMA2, exp2 (SFU; with POLY, every fourth pair on the FMA
-        // pipe), row-sum FADD2, bf16 pack, TMEM store; masked columns are
-        // -inf and give 0; chunks past the prefix are not read by P V
+        // p = 2^(s*scale*log2e - m) in four 32-column chunks: FFMA2, exp2
+        // (SFU; with POLY, every fourth pair on the FMA pipe), row-sum FADD2,
+        // bf16 pack, TMEM store; masked columns are -inf and give 0 (chunks
+        // past a short block's prefix are computed all the same: a branch
+        // between chunks costs more than it saves)
         {
           const float2 nm2 = make_float2(-m_use, -m_use);
           float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                             make_float2(0.f, 0.f)};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            if (32 * q >= nv) break;
             float2 pe[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c)

@@ -35,6 +35,9 @@ def _mixed_small():
 CASES = [
     _wl("ragged-2x8x8", 6, 20, 28, 2, 128, "bf16", (2, 8, 8)),
     _wl("ragged-d64", 5, 19, 23, 2, 64, "bf16", (2, 8, 8), tau=0.8),
+    # every edge case of a 2x8x8 block (t, y, x and their combinations), with
+    # valid-token counts that are not multiples of 16 (24, 42, 21, ...)
+    _wl("ragged-all-edges-d128", 5, 19, 23, 3, 128, "bf16", (2, 8, 8), tau=0.85),
     _wl("text-200", 4, 16, 24, 2, 128, "bf16", (2, 8, 8), text=200),
     _wl("tau1-dense-equivalent", 3, 16, 17, 2, 128, "bf16", (2, 8, 8), tau=1.0),
     _wl("one-block", 1, 4, 4, 2, 128, "bf16", (2, 8, 8)),
