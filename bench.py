@@ -373,7 +373,9 @@ def main(argv=None):
     ap.add_argument("--tau", type=float, default=0.9)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-chunk", type=int, default=8, help="heads per pipelined group in the e2e call")
+    ap.add_argument("--e2e-chunk", type=int, default=4, help="heads per pipelined group in the e2e call")
+    ap.add_argument("--e2e-slots", type=int, default=3, help="device group slots in the e2e call")
+    ap.add_argument("--e2e-streams", type=int, default=2, help="compute streams in the e2e call")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -511,7 +513,8 @@ def main(argv=None):
         oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
 
         def e2e_step():
-            api.grouped_attn_from_host(qh, kh, vh, oh, schemes, table, wl.text_tokens, head_chunk=args.e2e_chunk)
+            api.grouped_attn_from_host(qh, kh, vh, oh, schemes, table, wl.text_tokens, head_chunk=args.e2e_chunk,
+                                       slots=args.e2e_slots, compute_streams=args.e2e_streams)
         e2e_step()
         torch.cuda.synchronize()
         if world > 1:
@@ -527,7 +530,8 @@ def main(argv=None):
         extra["e2e"] = {"value": world * flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
                         "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                         "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": ems,
-                        "call": f"grouped_attn_from_host (pinned host tensors, head groups of {args.e2e_chunk})"}
+                        "call": f"grouped_attn_from_host (pinned host tensors, head groups of {args.e2e_chunk}, "
+                                f"{args.e2e_slots} device slots, {args.e2e_streams} compute streams)"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         extra["cpu_baseline"] = cpu_baseline(wl, q, k, v, flops)

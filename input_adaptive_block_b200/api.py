@@ -206,29 +206,44 @@ def grouped_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, schemes, tab
 
 
 def grouped_attn_from_host(qh: torch.Tensor, kh: torch.Tensor, vh: torch.Tensor, out_h: torch.Tensor, schemes,
-                           table, text_tokens: int = 0, head_chunk: int = 8, device=None,
-                           summary=("mean", "mean")) -> torch.Tensor:
+                           table, text_tokens: int = 0, head_chunk: int = 4, device=None,
+                           summary=("mean", "mean"), slots: int = 3, compute_streams: int = 2) -> torch.Tensor:
     """One layer from host memory to host memory, pipelined by head groups.
 
     qh, kh, vh, out_h: host tensors [N (+text), heads, d] (pinned for the
     copies to overlap).  Heads are independent in every step, so the layer
-    is streamed through the GPU in groups of head_chunk heads: the copy
+    is streamed through the GPU in groups of head_chunk heads: an upload
     stream brings group g in (strided 2-D copies, spade_copy_head_slice)
-    while the compute stream runs the grouped launch on group g-1 and the
-    copy stream returns finished groups.  Device buffers: two group slots.
-    Returns out_h after the call's work is enqueued; the caller synchronises
-    (or waits on the current stream, which this call joins at the end)."""
+    while the compute stream runs the grouped launch on an earlier group and
+    a download stream returns finished groups (uploads and downloads use the
+    two directions of the link at once).  Consecutive groups alternate over
+    `compute_streams` compute streams, so a group's kernels can start on the
+    SMs that the previous group's attention launch has already released.
+    Device buffers: `slots` group slots of Q, K, V and O; group g reuses slot
+    g % slots once group g - slots is back on the host.  Returns out_h after the call's work is
+    enqueued; the caller synchronises (or waits on the current stream, which
+    this call joins at the end)."""
+    if slots < 2:
+        raise ValueError("slots must be >= 2")
+    if compute_streams < 1 or compute_streams > slots:
+        raise ValueError("compute_streams must be in 1..slots")
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     rows, heads, d = qh.shape
     dt = dtype_code(qh.dtype)
     lib = _lib.load()
-    compute = torch.cuda.current_stream(dev)
-    copy = torch.cuda.Stream(dev)
+    caller = torch.cuda.current_stream(dev)
+    computes = [caller] + [torch.cuda.Stream(dev) for _ in range(compute_streams - 1)]
+    for c in computes[1:]:
+        c.wait_stream(caller)
+    up = torch.cuda.Stream(dev)
+    down = torch.cuda.Stream(dev)
     groups = [(h0, min(head_chunk, heads - h0)) for h0 in range(0, heads, head_chunk)]
     hcmax = max(hc for _, hc in groups)
-    # two slots x (q, k, v, out), each a flat buffer viewed as [rows, hc, d] for the group it holds
-    slots = [[torch.empty(rows * hcmax * d, dtype=qh.dtype, device=dev) for _ in range(4)] for _ in range(2)]
-    ws = [None, None]
+    ns = min(slots, len(groups))
+    # slot x (q, k, v, out), each a flat buffer viewed as [rows, hc, d] for the group it holds
+    bufs = [[torch.empty(rows * hcmax * d, dtype=qh.dtype, device=dev) for _ in range(4)] for _ in range(ns)]
+    need = max(grouped_workspace_bytes(schemes, list(table[h0: h0 + hc]), d, text_tokens) for h0, hc in groups)
+    wss = [torch.empty(max(need, 256), dtype=torch.uint8, device=dev) for _ in computes]   # one per compute stream
     loaded = [torch.cuda.Event() for _ in groups]
     done = [torch.cuda.Event() for _ in groups]
     returned = [torch.cuda.Event() for _ in groups]
@@ -238,35 +253,32 @@ def grouped_attn_from_host(qh: torch.Tensor, kh: torch.Tensor, vh: torch.Tensor,
 
     def load(gi):
         h0, hc = groups[gi]
-        buf = slots[gi % 2]
-        if gi >= 2:
-            copy.wait_event(returned[gi - 2])             # the slot's previous group is back on the host
-        for src, dstb in zip((qh, kh, vh), buf[:3]):
+        if gi >= ns:
+            up.wait_event(returned[gi - ns])              # the slot's previous group is back on the host
+        for src, dstb in zip((qh, kh, vh), bufs[gi % ns][:3]):
             check(lib.spade_copy_head_slice(dstb.data_ptr(), host_ptr(src), rows, heads, h0, hc, d, dt, 1,
-                                            copy.cuda_stream), "spade_copy_head_slice")
-        loaded[gi].record(copy)
+                                            up.cuda_stream), "spade_copy_head_slice")
+        loaded[gi].record(up)
 
-    with torch.cuda.stream(copy):
-        load(0)
+    for gi in range(ns - 1):
+        load(gi)
     for gi, (h0, hc) in enumerate(groups):
-        if gi + 1 < len(groups):
-            with torch.cuda.stream(copy):
-                load(gi + 1)
-        buf = slots[gi % 2]
+        if gi + ns - 1 < len(groups):
+            load(gi + ns - 1)
+        compute = computes[gi % len(computes)]
         compute.wait_event(loaded[gi])
-        q, k, v, o = (b[: rows * hc * d].view(rows, hc, d) for b in buf)
-        rows_t = list(table[h0: h0 + hc])
-        need = grouped_workspace_bytes(schemes, rows_t, d, text_tokens)
-        if ws[gi % 2] is None or ws[gi % 2].numel() < need:
-            ws[gi % 2] = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-        out = grouped_attn(q, k, v, schemes, rows_t, text_tokens, out=o, workspace=ws[gi % 2], stream=compute,
-                           summary=summary)
+        q, k, v, o = (b[: rows * hc * d].view(rows, hc, d) for b in bufs[gi % ns])
+        out = grouped_attn(q, k, v, schemes, list(table[h0: h0 + hc]), text_tokens, out=o,
+                           workspace=wss[gi % len(computes)], stream=compute, summary=summary)
         done[gi].record(compute)
-        copy.wait_event(done[gi])
+        down.wait_event(done[gi])
         check(lib.spade_copy_head_slice(out.data_ptr(), host_ptr(out_h), rows, heads, h0, hc, d, dt, 0,
-                                        copy.cuda_stream), "spade_copy_head_slice")
-        returned[gi].record(copy)
-    compute.wait_stream(copy)
+                                        down.cuda_stream), "spade_copy_head_slice")
+        returned[gi].record(down)
+    for c in computes[1:]:
+        caller.wait_stream(c)
+    caller.wait_stream(down)
+    caller.wait_stream(up)
     return out_h
 
 

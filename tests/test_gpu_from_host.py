@@ -10,8 +10,8 @@ from spade_workloads import Scheme, Workload, make_qkv
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("chunk,text", [(2, 0), (3, 0), (4, 64)])
-def test_from_host_equals_device_call(chunk, text):
+@pytest.mark.parametrize("chunk,text,slots,streams", [(2, 0, 3, 2), (3, 0, 2, 1), (4, 64, 3, 2), (1, 0, 4, 3)])
+def test_from_host_equals_device_call(chunk, text, slots, streams):
     T, H, W, heads = 5, 16, 24, 6
     wl = Workload("from-host", 61, T, H, W, heads, 128, "bf16", text, (Scheme(T, H, W, 2, 8, 8),),
                   (0,) * heads, (0.85, 0.9, 0.95, 0.85, 0.9, 0.95), (False,) * heads)
@@ -21,7 +21,8 @@ def test_from_host_equals_device_call(chunk, text):
     ref = api.grouped_attn(q, k, v, schemes, table, text)
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
     oh = torch.empty(qh.shape, dtype=qh.dtype).pin_memory()
-    api.grouped_attn_from_host(qh, kh, vh, oh, schemes, table, text, head_chunk=chunk)
+    api.grouped_attn_from_host(qh, kh, vh, oh, schemes, table, text, head_chunk=chunk, slots=slots,
+                               compute_streams=streams)
     torch.cuda.synchronize()
     assert api.last_device_status() == 0
     assert torch.equal(oh, ref.cpu())
