@@ -14,9 +14,9 @@
 //    zero-filled by the TMA unit.  Key/value blocks clipped by the grid edge
 //    are loaded with a box of their own clipped extents (one map per edge
 //    case), so their valid tokens form a prefix of the tile: the score MMA's
-//    N, the P V MMA's K and the exponentials all stop at that prefix (rounded
-//    up to 16) instead of computing padded columns.  No tiled copy of Q/K/V is
-//    ever written.
+//    N and the P V MMA's K stop at that prefix (rounded up to 16) instead of
+//    computing padded columns, and the softmax masks the columns past it.  No
+//    tiled copy of Q/K/V is ever written.
 //  * tcgen05.mma (kind::f16, bf16 in, fp32 accumulate), issued by one thread.
 //    TMEM (512 columns): S0 | S1 | S2 (fp32 scores; key block g of the CTA
 //    uses buffer g % 3) | O (fp32).  The softmax reads S(g) into registers and
@@ -460,13 +460,13 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------- MMA issuers --
-    // Warp 1 issues the score MMAs S(k) = Q K_k^T, warp 2 the P V(j) MMAs.
-    // The two streams touch disjoint TMEM (S buffers vs P buffers and O) and
-    // each commit tracks only its own warp's MMAs, so each warp blocks only on
-    // its own events: S(k) waits for its K tile and for the group that owns
-    // S buffer k % 2 to have read S(k-2); P V(j) waits for P(j) and V_j.  One
-    // warp waiting never holds back the other's issue, which keeps the
-    // (shallow) tensor instruction queue fed.  Each warp runs in uniform
+    // Warp 1 issues the score MMAs S(g) = Q K_g^T, warp 2 the P V(g) MMAs.
+    // Each commit tracks only its own warp's MMAs, so each warp blocks only on
+    // its own events: S(g) waits for its K tile and for P V(g-3) to have
+    // completed (buffer g % 3 then no longer holds P(g-3)); P V(g) waits for
+    // P(g) and V_g.  One warp waiting never holds back the other's issue,
+    // which keeps the (shallow) tensor instruction queue fed; a single issuer
+    // in a fixed order measured 23 % slower.  Each warp runs in uniform
     // control flow; one elected lane issues each tcgen05.mma / commit.
     //
     // Ring positions inside an item with n blocks (base B): K_k at B + k for
