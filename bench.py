@@ -228,32 +228,33 @@ def cpu_baseline(wl, q, k, v, total_flops, budget_heads=4, qblocks=24):
 
 def selection_timing(api, q, k, wl, steps, stream, hbm_gbs):
     """Steps 1-4 timed one stage at a time through the public C ABI on the
-    bench workload (single scheme): summarize Q, summarize K, estimate,
-    select.  L2 is flushed (a 256 MB write) before every timed call, so each
-    stage reads its inputs from HBM.  Algorithmic bytes: summarize reads one
-    [N, heads, d] tensor and writes [heads, nb, d] fp32 means; estimate reads
-    both means and writes [heads, nb, nb] fp32 probabilities (plus
-    2 nb^2 d heads FLOPs); select reads the probabilities and writes the
-    counts and the kept ids."""
+    bench workload (single scheme), in the form the grouped call runs them:
+    summarize Q and K (one launch, spade_summarize_qk), the estimator's pooled scores
+    (spade_estimate_scores), and the index search with the softmax fused in
+    (spade_select_scores).  L2 is flushed (a 256 MB write) before every
+    timed call, so each stage reads its inputs from HBM.  Algorithmic bytes:
+    summarize reads the two [N, heads, d] tensors and writes two
+    [heads, nb, d] fp32 means; the estimator reads both means and writes [heads, nb, nb] fp32
+    scores (plus 2 nb^2 d heads FLOPs); the index search reads the scores and
+    writes the counts and the kept ids."""
     import torch
     sc = wl.schemes[0]
     g = sc.as_tuple()
     nb, heads, d = sc.nb, wl.heads, wl.d
     esz = q.element_size()
-    qm = api.summarize(q, g)
-    km = api.summarize(k, g)
-    prob = api.estimate(qm, km)
-    cnt, idx = api.select(prob, wl.head_tau)
+    qm, km = api.summarize_qk(q, k, g)
+    scores = api.estimate_scores(qm, km)
+    cnt, idx = api.select_scores(scores, wl.head_tau)
     torch.cuda.synchronize()
     kept_ids = int(cnt.sum().item())
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=q.device)
     stages = {
-        "summarize_q": (lambda: api.summarize(q, g, out=qm), wl.N * heads * d * esz + nb * heads * d * 4, 0),
-        "summarize_k": (lambda: api.summarize(k, g, out=km), wl.N * heads * d * esz + nb * heads * d * 4, 0),
-        "estimate": (lambda: api.estimate(qm, km, out=prob), 2 * nb * heads * d * 4 + nb * nb * heads * 4,
+        "summarize_qk": (lambda: api.summarize_qk(q, k, g, qout=qm, kout=km),
+                         2 * (wl.N * heads * d * esz + nb * heads * d * 4), 0),
+        "estimate": (lambda: api.estimate_scores(qm, km, out=scores), 2 * nb * heads * d * 4 + nb * nb * heads * 4,
                      2 * nb * nb * d * heads),
-        "select": (lambda: api.select(prob, wl.head_tau, cnt=cnt, idx=idx), nb * nb * heads * 4 + nb * heads * 4
-                   + kept_ids * 4, 0),
+        "select": (lambda: api.select_scores(scores, wl.head_tau, cnt=cnt, idx=idx), nb * nb * heads * 4
+                   + nb * heads * 4 + kept_ids * 4, 0),
     }
     out = {}
     tot_ms, tot_bytes = 0.0, 0
@@ -501,7 +502,7 @@ def main(argv=None):
         hs = [h for h in range(wl.heads) if wl.head_scheme[h] == s_id and not wl.head_dense[h]]
         if hs:
             runs = 1 + sum(1 for a, b in zip(hs, hs[1:]) if b != a + 1)
-            n_runs += 2 * runs + 2
+            n_runs += runs + 2          # one Q+K summarize launch per run of heads, scores, select
     extra["gpu_launches"] = args.steps * (n_runs + 2)
     extra["clocks"] = clocks
 

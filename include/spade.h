@@ -95,6 +95,13 @@ spade_status spade_tile3d(const void* x, void* xt, spade_geom g, int heads, int 
 spade_status spade_summarize(const void* x, float* xmean, spade_geom g, int heads, int d,
                              spade_dtype dt, spade_stream_t stream);
 
+/* spade_summarize of Q and of K in one launch (the form spade_grouped_attn
+ * runs): qmean from q and kmean from k, each exactly as spade_summarize
+ * computes it.  q, k: [>= N, heads, d] token order, dtype `dt`; qmean,
+ * kmean: [heads, nb, d] float32. */
+spade_status spade_summarize_qk(const void* q, const void* k, float* qmean, float* kmean, spade_geom g,
+                                int heads, int d, spade_dtype dt, spade_stream_t stream);
+
 /* The same pass with another of the Summarizer's reduces: mode
  * SPADE_SUM_MAX / SPADE_SUM_MIN give the elementwise max / min over each
  * block's valid tokens (exact: no rounding), SPADE_SUM_MEAN is
@@ -110,12 +117,27 @@ spade_status spade_summarize_mode(const void* x, float* out, spade_geom g, int h
 spade_status spade_estimate(const float* qmean, const float* kmean, float* prob,
                             int heads, int nb, int d, spade_stream_t stream);
 
+/* Step 3 without its softmax: scores[h,i,j] = qmean[h,i,:] . kmean[h,j,:] /
+ * sqrt(d), float32, computed exactly as spade_estimate computes them before
+ * its softmax (split-precision TF32 on the tensor cores, fp32-level
+ * accuracy).  This is the form spade_grouped_attn runs: the softmax is then
+ * formed by spade_select_scores as it reads each row, so the probabilities
+ * never pass through memory.  Same arguments and limits as spade_estimate;
+ * returns SPADE_ERR_UNSUPPORTED where the driver's tensor-map encoder is
+ * unavailable (spade_estimate then falls back to a CUDA-core kernel). */
+spade_status spade_estimate_scores(const float* qmean, const float* kmean, float* scores,
+                                   int heads, int nb, int d, spade_stream_t stream);
+
 /* ---- step 4: index search -----------------------------------------------
  * Abstract, executor "low-overhead index search"; Methodology 3, ranked
  * block-sparse representation.  Per (head h, query block i): kept set = {i},
  * then other blocks in descending prob (ties -> lower id) until the mass
  * (prob[h,i,i] + sum of added) >= tau[h]; tau >= 1 or a mass that never
- * reaches tau keeps every block.  Computed in float32.
+ * reaches tau keeps every block.  Probabilities are compared as float32;
+ * masses are summed in fixed point (units of 2^-30, or of 2^-30 times the
+ * row sum when a row sums to more than 1), so every sum is exact and the
+ * result does not depend on summation order.  Entries are clamped to [0, 1]
+ * (NaN counts as 0).
  * prob    : [heads, nb, nb] float32 (device).
  * tau_host: [heads] float32 HOST array, read during the call.
  * cnt     : [heads, nb] int32 out, number of kept blocks (>= 1).
@@ -124,6 +146,14 @@ spade_status spade_estimate(const float* qmean, const float* kmean, float* prob,
  * Limits: nb <= 1024, heads <= 1024. */
 spade_status spade_select(const float* prob, const float* tau_host, int* cnt, int* idx,
                           int heads, int nb, spade_stream_t stream);
+
+/* Steps 3 and 4 fused: the Estimator's softmax over each row of `scores`
+ * (from spade_estimate_scores: prob = exp(s - max) / sum, float32) followed
+ * by the same index search as spade_select, in one pass over the row.
+ * scores: [heads, nb, nb] float32 (device); other arguments, outputs and
+ * limits as spade_select. */
+spade_status spade_select_scores(const float* scores, const float* tau_host, int* cnt, int* idx,
+                                 int heads, int nb, spade_stream_t stream);
 
 /* Static windows merged with dynamic selection (Methodology 2, Policy
  * Application: "balancing static windows and dynamic selection").  The

@@ -28,8 +28,12 @@ class SpadeHeadScheme(ctypes.Structure):
 SIGNATURES = {
     "spade_tile3d": (c_int, [c_void_p, c_void_p, SpadeGeom, c_int, c_int, c_int, c_void_p]),
     "spade_summarize": (c_int, [c_void_p, c_void_p, SpadeGeom, c_int, c_int, c_int, c_void_p]),
+    "spade_summarize_qk": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, SpadeGeom, c_int, c_int, c_int,
+                                   c_void_p]),
     "spade_estimate": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
+    "spade_estimate_scores": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p]),
     "spade_select": (c_int, [c_void_p, POINTER(c_float), c_void_p, c_void_p, c_int, c_int, c_void_p]),
+    "spade_select_scores": (c_int, [c_void_p, POINTER(c_float), c_void_p, c_void_p, c_int, c_int, c_void_p]),
     "spade_attn_workspace_bytes": (c_size_t, [SpadeGeom, c_int, c_int, c_int]),
     "spade_block_sparse_attn": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                         SpadeGeom, c_int, c_int, c_int, c_int, c_void_p, c_size_t,

@@ -15,7 +15,8 @@ from . import _lib
 from ._lib import SpadeGeom, SpadeHeadScheme, check
 
 __all__ = [
-    "geom", "dtype_code", "tile3d", "summarize", "estimate", "select", "attn_workspace_bytes",
+    "geom", "dtype_code", "tile3d", "summarize", "summarize_qk", "estimate", "estimate_scores", "select", "select_scores",
+    "attn_workspace_bytes",
     "block_sparse_attn", "block_sparse_attn_noalloc", "grouped_workspace_bytes", "grouped_attn", "grouped_head_lists",
     "last_device_status", "selftest_bounded_wait", "num_blocks", "sics_workspace_bytes", "sics", "select_window",
     "grouped_attn_from_host",
@@ -85,6 +86,23 @@ def summarize(x: torch.Tensor, g, out: Optional[torch.Tensor] = None, stream=Non
     return out
 
 
+def summarize_qk(q: torch.Tensor, k: torch.Tensor, g, qout: Optional[torch.Tensor] = None,
+                 kout: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Block means of Q and of K in one launch."""
+    gg = geom(g)
+    heads, d = q.shape[1], q.shape[2]
+    if k.shape[1:] != q.shape[1:] or k.dtype != q.dtype:
+        raise ValueError("q and k must have the same heads, d and dtype")
+    nb = num_blocks(gg)
+    if qout is None:
+        qout = torch.empty(heads, nb, d, dtype=torch.float32, device=q.device)
+    if kout is None:
+        kout = torch.empty(heads, nb, d, dtype=torch.float32, device=q.device)
+    check(_lib.load().spade_summarize_qk(_dev(q, "q"), _dev(k, "k"), _dev(qout, "qmean"), _dev(kout, "kmean"),
+                                         gg, heads, d, dtype_code(q.dtype), _stream(stream)), "spade_summarize_qk")
+    return qout, kout
+
+
 def estimate(qmean: torch.Tensor, kmean: torch.Tensor, out: Optional[torch.Tensor] = None,
              stream=None) -> torch.Tensor:
     heads, nb, d = qmean.shape
@@ -95,17 +113,38 @@ def estimate(qmean: torch.Tensor, kmean: torch.Tensor, out: Optional[torch.Tenso
     return out
 
 
+def estimate_scores(qmean: torch.Tensor, kmean: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """The Estimator's pooled scores Qbar . Kbar^T / sqrt(d) (no softmax)."""
+    heads, nb, d = qmean.shape
+    if out is None:
+        out = torch.empty(heads, nb, nb, dtype=torch.float32, device=qmean.device)
+    check(_lib.load().spade_estimate_scores(_dev(qmean, "qmean"), _dev(kmean, "kmean"), _dev(out, "scores"),
+                                            heads, nb, d, _stream(stream)), "spade_estimate_scores")
+    return out
+
+
+def _select(fn_name: str, x: torch.Tensor, taus: Sequence[float], cnt, idx, stream):
+    heads, nb, _ = x.shape
+    if cnt is None:
+        cnt = torch.empty(heads, nb, dtype=torch.int32, device=x.device)
+    if idx is None:
+        idx = torch.full((heads, nb, nb), -1, dtype=torch.int32, device=x.device)
+    tau_arr = (ctypes.c_float * heads)(*[float(t) for t in taus])
+    check(getattr(_lib.load(), fn_name)(_dev(x, "input"), tau_arr, _dev(cnt, "cnt"), _dev(idx, "idx"),
+                                        heads, nb, _stream(stream)), fn_name)
+    return cnt, idx
+
+
 def select(prob: torch.Tensor, taus: Sequence[float], cnt: Optional[torch.Tensor] = None,
            idx: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    heads, nb, _ = prob.shape
-    if cnt is None:
-        cnt = torch.empty(heads, nb, dtype=torch.int32, device=prob.device)
-    if idx is None:
-        idx = torch.full((heads, nb, nb), -1, dtype=torch.int32, device=prob.device)
-    tau_arr = (ctypes.c_float * heads)(*[float(t) for t in taus])
-    check(_lib.load().spade_select(_dev(prob, "prob"), tau_arr, _dev(cnt, "cnt"), _dev(idx, "idx"),
-                                   heads, nb, _stream(stream)), "spade_select")
-    return cnt, idx
+    return _select("spade_select", prob, taus, cnt, idx, stream)
+
+
+def select_scores(scores: torch.Tensor, taus: Sequence[float], cnt: Optional[torch.Tensor] = None,
+                  idx: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Softmax of each score row fused with the index search."""
+    return _select("spade_select_scores", scores, taus, cnt, idx, stream)
 
 
 def select_window(prob: torch.Tensor, taus: Sequence[float], radius, g, cnt: Optional[torch.Tensor] = None,

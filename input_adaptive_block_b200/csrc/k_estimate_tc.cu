@@ -1,8 +1,10 @@
-// Step 3 on the tensor cores: the Estimator
-//   prob[h,i,:] = softmax_j( qmean[h,i,:] . kmean[h,j,:] / sqrt(d) )
+// Step 3 on the tensor cores: the Estimator's pooled scores
+//   score[h,i,j] = qmean[h,i,:] . kmean[h,j,:] / sqrt(d)
+// and, for the standalone estimator, their softmax over j
 // (SPADE technical summary (gist.science/paper/2608.03335), Methodology 1,
 // "Summarizer & Estimator Expressions": inter-block importance from the
-// block summaries).
+// block summaries).  On the grouped path the softmax is formed by the index
+// search as it reads each row (k_select.cu), so only the scores are written.
 //
 // The block means are fp32 and the scores decide the kept sets, so the
 // contraction keeps fp32-level accuracy with error-compensated split
@@ -11,17 +13,16 @@
 // (exact in fp32), and S = Qhi Khi^T + Qhi Klo^T + Qlo Khi^T (the lo lo term
 // and the TF32 rounding of lo are below 2^-20 relative).
 //
-//  * Persistent CTAs over items (head, 128 query rows).  Per item, per
-//    128-column key tile, per 32-element d chunk: TMA loads the fp32 Q and K
-//    chunks (128 rows x 128 B, 128-byte swizzled: the K-major layout the MMA
-//    reads); a converter warpgroup rewrites each chunk as hi in place and lo
-//    beside it (the split is elementwise, so the swizzled layout carries
-//    over); one thread issues the 12 tcgen05.mma (kind::tf32, M=N=128, K=8)
-//    of the chunk into one of two S tiles in TMEM.
-//  * An epilogue warpgroup (thread = query row) reads each finished S tile
-//    with tcgen05.ld, scales it, keeps a running row max and sum (online
-//    softmax over the key tiles), stages the scores in the output row, and
-//    after the last tile rewrites its row as probabilities.
+//  * Persistent CTAs over items (head, 128 query rows, 128 key columns),
+//    dealt round-robin, so the work is spread evenly over the SMs.  Per item
+//    and 32-element d chunk: TMA loads the fp32 Q and K chunks (128 rows x
+//    128 B, 128-byte swizzled: the K-major layout the MMA reads); a converter
+//    warpgroup rewrites each chunk as hi in place and lo beside it (the split
+//    is elementwise, so the swizzled layout carries over); one thread issues
+//    the 12 tcgen05.mma (kind::tf32, M=128, K=8, N = the item's valid key
+//    columns rounded up to 16) into one of two S tiles in TMEM.
+//  * Two epilogue warpgroups (64 columns each; thread = query row) read a
+//    finished tile with tcgen05.ld, release it, scale it and store it.
 //  * Every wait is bounded (globaltimer); a timeout latches SPADE_ERR_TIMEOUT
 //    in the device status word and the CTA winds down.
 #include <cudaTypedefs.h>
@@ -35,12 +36,12 @@ namespace {
 constexpr int kStages = 3;
 constexpr int kChunk = 128 * 128;           // 128 rows x 128 B (32 fp32 of d)
 constexpr int kStageBytes = 4 * kChunk;     // Q hi, Q lo, K hi, K lo
-constexpr int kThreads = 384;               // producer, MMA, 2 idle, converters (4 warps), epilogue (4 warps)
+constexpr int kThreads = 512;               // producer, MMA, 2 idle, converters (4 warps), 2 x epilogue (4 warps)
 constexpr int kSmem = kStages * kStageBytes + 256 + 1024;
 
 struct __align__(64) EstTcParams {
   CUtensorMap tm_q, tm_k;   // [heads][nb][d] fp32: dims {d, nb, heads}, box {32, 128, 1}
-  float* prob;              // [heads][nb][nb]
+  float* out;               // [heads][nb][nb] scores
   int nb, d, nrt, n_items;
   float scale;
   int* status;
@@ -79,7 +80,9 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t saddr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 // kind::tf32: D fp32 (bit 4), A and B TF32 (format 2 in bits 7 and 10), K-major, N >> 3, M >> 4.
-constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+__device__ __forceinline__ uint32_t idesc_tf32(uint32_t n) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
+}
 
 __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_constant__ EstTcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -89,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
   uint64_t* conv = bars + kStages;         // [kStages] split into hi / lo (128 threads)
   uint64_t* empty = bars + 2 * kStages;    // [kStages] MMAs done with the stage
   uint64_t* s_full = bars + 3 * kStages;   // [2] S tile complete
-  uint64_t* s_free = s_full + 2;           // [2] S tile read (128 threads)
+  uint64_t* s_free = s_full + 2;           // [2] S tile read (256 epilogue threads)
   uint64_t* fin = s_full + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -103,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&s_full[b], 1);
-      ptx::mbar_init(&s_free[b], 128);
+      ptx::mbar_init(&s_free[b], 256);
     }
     ptx::mbar_init(fin, 1);
     *abort_flag = 0;
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const EWaiter W{abort_flag, p.status, p.timeout_ns};
-  const int nct = p.nrt;          // key tiles = query tiles (both cover nb in 128s)
+  const int nt = p.nrt;           // key tiles = query tiles (both cover nb in 128s)
   const int ndc = p.d / 32;
 
   if (warp == 0) {
@@ -130,17 +133,17 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     uint32_t g = 0;
     bool ok = true;
     for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
-      const int h = it / p.nrt, rt = it - h * p.nrt;
-      for (int ct = 0; ok && ct < nct; ++ct)
-        for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
-          const int s = (int)(g % kStages);
-          ok = __all_sync(0xffffffffu, ewait(&empty[s], ((g / kStages) & 1) ^ 1, W));
-          if (!ok) break;
-          uint8_t* st = smem + s * kStageBytes;
-          ptx::mbar_arrive_expect_tx_elect(&full[s], 2 * kChunk);
-          ptx::tma_load_3d_elect(st, &p.tm_q, &full[s], 32 * dc, 128 * rt, h);
-          ptx::tma_load_3d_elect(st + 2 * kChunk, &p.tm_k, &full[s], 32 * dc, 128 * ct, h);
-        }
+      const int h = it / (nt * nt), rem = it - h * nt * nt;
+      const int rt = rem / nt, ct = rem - rt * nt;
+      for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
+        const int s = (int)(g % kStages);
+        ok = __all_sync(0xffffffffu, ewait(&empty[s], ((g / kStages) & 1) ^ 1, W));
+        if (!ok) break;
+        uint8_t* st = smem + s * kStageBytes;
+        ptx::mbar_arrive_expect_tx_elect(&full[s], 2 * kChunk);
+        ptx::tma_load_3d_elect(st, &p.tm_q, &full[s], 32 * dc, 128 * rt, h);
+        ptx::tma_load_3d_elect(st + 2 * kChunk, &p.tm_k, &full[s], 32 * dc, 128 * ct, h);
+      }
     }
     if (lane == 0 && !ok && g > 0) {   // wind down: let the loads issued land
       for (uint32_t k = (g > (uint32_t)kStages ? g - kStages : 0); k < g; ++k)
@@ -148,33 +151,34 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer --
-    uint32_t g = 0, gct = 0;
+    uint32_t g = 0, gi = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
-      for (int ct = 0; ok && ct < nct; ++ct, ++gct) {
-        const int b = (int)(gct & 1);
-        ok = __all_sync(0xffffffffu, ewait(&s_free[b], ((gct >> 1) & 1) ^ 1, W));
+    for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++gi) {
+      const int ct = (it % (nt * nt)) % nt;
+      const int nv = p.nb - 128 * ct < 128 ? p.nb - 128 * ct : 128;   // valid key columns
+      const uint32_t idesc = idesc_tf32((uint32_t)((nv + 15) & ~15));
+      const int b = (int)(gi & 1);
+      ok = __all_sync(0xffffffffu, ewait(&s_free[b], ((gi >> 1) & 1) ^ 1, W));
+      if (!ok) break;
+      const uint32_t ts = tmem + 128 * b;
+      for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
+        const int s = (int)(g % kStages);
+        ok = __all_sync(0xffffffffu, ewait(&conv[s], (g / kStages) & 1, W));
         if (!ok) break;
-        const uint32_t ts = tmem + 128 * b;
-        for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
-          const int s = (int)(g % kStages);
-          ok = __all_sync(0xffffffffu, ewait(&conv[s], (g / kStages) & 1, W));
-          if (!ok) break;
-          ptx::tc_fence_after();
-          const uint32_t base = ptx::smem_u32(smem + s * kStageBytes);
-          const uint64_t qhi = kdesc(base), qlo = kdesc(base + kChunk);
-          const uint64_t khi = kdesc(base + 2 * kChunk), klo = kdesc(base + 3 * kChunk);
+        ptx::tc_fence_after();
+        const uint32_t base = ptx::smem_u32(smem + s * kStageBytes);
+        const uint64_t qhi = kdesc(base), qlo = kdesc(base + kChunk);
+        const uint64_t khi = kdesc(base + 2 * kChunk), klo = kdesc(base + 3 * kChunk);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {           // 8 fp32 (32 B) of d per MMA
-            const uint64_t off = (uint64_t)((kk * 32) >> 4);
-            ptx::mma_ss_tf32_elect(ts, qhi + off, khi + off, kIdesc, (dc > 0 || kk > 0) ? 1u : 0u);
-            ptx::mma_ss_tf32_elect(ts, qhi + off, klo + off, kIdesc, 1u);
-            ptx::mma_ss_tf32_elect(ts, qlo + off, khi + off, kIdesc, 1u);
-          }
-          ptx::tc_commit_elect(&empty[s]);
+        for (int kk = 0; kk < 4; ++kk) {           // 8 fp32 (32 B) of d per MMA
+          const uint64_t off = (uint64_t)((kk * 32) >> 4);
+          ptx::mma_ss_tf32_elect(ts, qhi + off, khi + off, idesc, (dc > 0 || kk > 0) ? 1u : 0u);
+          ptx::mma_ss_tf32_elect(ts, qhi + off, klo + off, idesc, 1u);
+          ptx::mma_ss_tf32_elect(ts, qlo + off, khi + off, idesc, 1u);
         }
-        if (ok) ptx::tc_commit_elect(&s_full[b]);
+        ptx::tc_commit_elect(&empty[s]);
       }
+      if (ok) ptx::tc_commit_elect(&s_full[b]);
     }
     ptx::tc_commit_elect(fin);
     edrain(fin, 0, 100000000LL);
@@ -184,7 +188,6 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     uint32_t g = 0;
     bool ok = true;
     for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x)
-      for (int ct = 0; ok && ct < nct; ++ct)
         for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
           const int s = (int)(g % kStages);
           ok = ewait(&full[s], (g / kStages) & 1, W);
@@ -208,83 +211,41 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
           ptx::mbar_arrive(&conv[s]);
         }
   } else if (warp >= 8) {
-    // ---------------------------------------------------------- epilogue --
+    // --------------------------------------------------------- epilogues --
+    const int half = (warp - 8) >> 2;            // key columns 64*half .. 64*half + 63 of the tile
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const bool vec = (p.nb & 3) == 0;
-    uint32_t gct = 0;
+    uint32_t gi = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
-      const int h = it / p.nrt, rt = it - h * p.nrt;
+    for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++gi) {
+      const int h = it / (nt * nt), rem = it - h * nt * nt;
+      const int rt = rem / nt, ct = rem - rt * nt;
+      const int b = (int)(gi & 1);
+      ok = ewait(&s_full[b], (gi >> 1) & 1, W);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      ptx::tc_fence_after();
       const int i = 128 * rt + row;
-      float* prow = p.prob + ((long long)h * p.nb + (i < p.nb ? i : 0)) * p.nb;
-      float m = -INFINITY, l = 0.f;
-      for (int ct = 0; ct < nct; ++ct, ++gct) {
-        const int b = (int)(gct & 1);
-        ok = ewait(&s_full[b], (gct >> 1) & 1, W);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        ptx::tc_fence_after();
-        const int j0 = 128 * ct;
-        const int nv = p.nb - j0 < 128 ? p.nb - j0 : 128;   // valid key columns in this tile
-        // four 32-column pieces: scale, mask, fold into the running max / sum
-        // (online softmax), stage the scores in the output row
-#pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t sr[32];
-          ptx::tmem_ld32(tmem + lane_base + 128 * b + c0, sr);
-          float cm = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float v = c0 + c < nv ? __uint_as_float(sr[c]) * p.scale : -INFINITY;
-            sr[c] = __float_as_uint(v);
-            cm = fmaxf(cm, v);
-          }
-          if (cm > -INFINITY) {
-            const float mn = fmaxf(m, cm);
-            float cs = 0.f;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) cs += expf(__uint_as_float(sr[c]) - mn);
-            l = l * expf(m - mn) + cs;
-            m = mn;
-          }
-          if (i < p.nb) {
-            if (vec) {
-              float4* dst = reinterpret_cast<float4*>(prow + j0 + c0);
-#pragma unroll
-              for (int c4 = 0; c4 < 8; ++c4)
-                if (c0 + 4 * c4 < nv)
-                  dst[c4] = make_float4(__uint_as_float(sr[4 * c4]), __uint_as_float(sr[4 * c4 + 1]),
-                                        __uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3]));
-            } else {
-#pragma unroll
-              for (int c = 0; c < 32; ++c)
-                if (c0 + c < nv) prow[j0 + c0 + c] = __uint_as_float(sr[c]);
-            }
-          }
-        }
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&s_free[b]);
-      }
-      if (!ok) break;
-      if (i < p.nb) {
-        // probabilities: the thread rewrites its own staged row
-        const float inv = 1.0f / l;
+      const int j0 = 128 * ct + 64 * half;
+      const int nv = p.nb - j0 < 64 ? p.nb - j0 : 64;   // valid columns of this half (warp-uniform)
+      uint32_t sr[64];
+      if (nv > 0) ptx::tmem_ld64(tmem + lane_base + 128 * b + 64 * half, sr);
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&s_free[b]);                // the tile may be overwritten now
+      if (nv > 0 && i < p.nb) {
+        float* dst = p.out + ((long long)h * p.nb + i) * p.nb + j0;
         if (vec) {
-          float4* r4 = reinterpret_cast<float4*>(prow);
-          for (int c0 = 0; c0 < p.nb / 4; c0 += 16) {     // sixteen 16-byte loads in flight
-            float4 v[16];
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
-              if (c0 + u < p.nb / 4) v[u] = r4[c0 + u];
-#pragma unroll
-            for (int u = 0; u < 16; ++u)
-              if (c0 + u < p.nb / 4)
-                r4[c0 + u] = make_float4(expf(v[u].x - m) * inv, expf(v[u].y - m) * inv, expf(v[u].z - m) * inv,
-                                         expf(v[u].w - m) * inv);
-          }
+          for (int c4 = 0; c4 < 16; ++c4)
+            if (4 * c4 < nv)
+              reinterpret_cast<float4*>(dst)[c4] =
+                  make_float4(__uint_as_float(sr[4 * c4]) * p.scale, __uint_as_float(sr[4 * c4 + 1]) * p.scale,
+                              __uint_as_float(sr[4 * c4 + 2]) * p.scale, __uint_as_float(sr[4 * c4 + 3]) * p.scale);
         } else {
-          for (int c = 0; c < p.nb; ++c) prow[c] = expf(prow[c] - m) * inv;
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < nv) dst[c] = __uint_as_float(sr[c]) * p.scale;
         }
       }
     }
@@ -317,21 +278,60 @@ bool map_means(CUtensorMap* m, const float* base, int heads, int nb, int d) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row softmax in place, one warp per row (the standalone estimator's
+// probabilities from its scores): p_j = exp(s_j - max) / sum.
+template <int NPL>
+__global__ void __launch_bounds__(256) softmax_rows_kernel(float* __restrict__ s, long long rows, int nb) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  float* r = s + row * nb;
+  float v[NPL];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < NPL; ++e) {
+    const int j = lane + 32 * e;
+    v[e] = j < nb ? r[j] : -INFINITY;
+    mx = fmaxf(mx, v[e]);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float l = 0.f;
+#pragma unroll
+  for (int e = 0; e < NPL; ++e) {
+    v[e] = lane + 32 * e < nb ? expf(v[e] - mx) : 0.f;
+    l += v[e];
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  const float inv = 1.0f / l;
+#pragma unroll
+  for (int e = 0; e < NPL; ++e)
+    if (lane + 32 * e < nb) r[lane + 32 * e] = v[e] * inv;
+}
+
+template <int NPL>
+cudaError_t launch_softmax_rows(float* s, long long rows, int nb, cudaStream_t st) {
+  const long long blocks = (rows + 7) / 8;
+  softmax_rows_kernel<NPL><<<(unsigned)blocks, 256, 0, st>>>(s, rows, nb);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
-cudaError_t launch_estimate_tc(const float* qm, const float* km, float* prob, int heads, int nb, int d, int* status,
-                               cudaStream_t s) {
+cudaError_t launch_estimate_tc(const float* qm, const float* km, float* out, int heads, int nb, int d, int* status,
+                               bool probs, cudaStream_t s) {
   if (!encode_fn()) return cudaErrorNotSupported;
   if (d % 32 != 0 || (reinterpret_cast<uintptr_t>(qm) & 15) || (reinterpret_cast<uintptr_t>(km) & 15))
     return cudaErrorInvalidValue;
   static EstTcParams tp;
   memset(&tp, 0, sizeof(tp));
   if (!map_means(&tp.tm_q, qm, heads, nb, d) || !map_means(&tp.tm_k, km, heads, nb, d)) return cudaErrorInvalidValue;
-  tp.prob = prob;
+  tp.out = out;
   tp.nb = nb;
   tp.d = d;
   tp.nrt = (nb + 127) / 128;
-  tp.n_items = heads * tp.nrt;
+  tp.n_items = heads * tp.nrt * tp.nrt;
   tp.scale = 1.0f / sqrtf((float)d);
   tp.status = status;
   tp.timeout_ns = device_wait_timeout_ns();
@@ -341,7 +341,13 @@ cudaError_t launch_estimate_tc(const float* qm, const float* km, float* prob, in
   const int grid = tp.n_items < num_sms() ? tp.n_items : num_sms();
   if (grid <= 0) return cudaSuccess;
   estimate_tc_kernel<<<grid, kThreads, kSmem, s>>>(tp);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !probs) return e;
+  const long long rows = (long long)heads * nb;
+  if (nb <= 256) return launch_softmax_rows<8>(out, rows, nb, s);
+  if (nb <= 512) return launch_softmax_rows<16>(out, rows, nb, s);
+  if (nb <= 1024) return launch_softmax_rows<32>(out, rows, nb, s);
+  return launch_softmax_rows<64>(out, rows, nb, s);
 }
 
 }  // namespace spade

@@ -73,8 +73,12 @@ __device__ __forceinline__ void accumulate(float (&acc)[BF16 ? 8 : 4], const uin
   }
 }
 
+// Two tensors (Q and K) can share one launch: units [0, n) read in0 into
+// out0, units [n, 2n) read in1 into out1 (in1 == nullptr: one tensor).
 template <bool BF16, int MODE>
-__global__ void __launch_bounds__(256, 5) summarize_kernel(const uint8_t* __restrict__ x, float* __restrict__ out,
+__global__ void __launch_bounds__(256, 5) summarize_kernel(const uint8_t* __restrict__ in0,
+                                                         const uint8_t* __restrict__ in1,
+                                                         float* __restrict__ out0, float* __restrict__ out1,
                                                          Geo g, long long row_bytes, int head_off_bytes,
                                                          int chunks, int d) {
   constexpr int EPC = BF16 ? 8 : 4;  // elements per 16-byte chunk
@@ -83,9 +87,14 @@ __global__ void __launch_bounds__(256, 5) summarize_kernel(const uint8_t* __rest
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   const int groups = (chunks + 31) / 32;
   const long long n_units = (long long)g.nb * groups;
+  const long long all_units = in1 ? 2 * n_units : n_units;
   const long long sy = (long long)g.W * row_bytes;     // next y row
   const long long st = (long long)g.H * sy;            // next frame
-  for (long long u = gwarp; u < n_units; u += nwarps) {
+  for (long long uu = gwarp; uu < all_units; uu += nwarps) {
+    const bool second = uu >= n_units;
+    const long long u = second ? uu - n_units : uu;
+    const uint8_t* x = second ? in1 : in0;
+    float* out = second ? out1 : out0;
     const int b = (int)(u / groups);
     const int c = (int)(u - (long long)b * groups) * 32 + lane;
     int t0, y0, x0, et, eh, ew;
@@ -148,32 +157,43 @@ cudaError_t launch_tile3d(const void* x, void* xt, const Geo& g, int heads, int 
   return cudaGetLastError();
 }
 
+// Grid: every warp takes the same number of (block, chunk group) units,
+// dealt round-robin, with all warps resident at once (5 CTAs of 8 warps per
+// SM): no partial last round of units while the rest of the GPU idles.
 template <int MODE>
-cudaError_t launch_summarize_m(const void* x, float* out, const Geo& g, int heads_total, int h0, int hc, int d,
-                               spade_dtype dt, cudaStream_t s) {
+cudaError_t launch_summarize_m(const void* x0, const void* x1, float* out0, float* out1, const Geo& g,
+                               int heads_total, int h0, int hc, int d, spade_dtype dt, cudaStream_t s) {
   const int esz = dt == SPADE_BF16 ? 2 : 4;
   const long long row_bytes = (long long)heads_total * d * esz;
   const int chunks = hc * d * esz / 16;
   const int groups = (chunks + 31) / 32;
-  const long long units = (long long)g.nb * groups;
-  long long blocks = (units + 7) / 8;                  // 8 warps per CTA
-  const long long cap = 5LL * num_sms();               // all resident: 40 warps per SM
-  if (blocks > cap) blocks = cap;
+  const long long units = (long long)g.nb * groups * (x1 ? 2 : 1);
+  const long long resident = 5LL * num_sms() * 8;      // warps
+  const long long per_warp = (units + resident - 1) / resident;
+  const long long warps = (units + per_warp - 1) / per_warp;
+  long long blocks = (warps + 7) / 8;
   if (blocks < 1) blocks = 1;
+  const uint8_t* a = static_cast<const uint8_t*>(x0);
+  const uint8_t* b = static_cast<const uint8_t*>(x1);
   if (dt == SPADE_BF16)
-    summarize_kernel<true, MODE><<<(int)blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), out, g, row_bytes,
-                                                              h0 * d * esz, chunks, d);
+    summarize_kernel<true, MODE><<<(int)blocks, 256, 0, s>>>(a, b, out0, out1, g, row_bytes, h0 * d * esz, chunks, d);
   else
-    summarize_kernel<false, MODE><<<(int)blocks, 256, 0, s>>>(static_cast<const uint8_t*>(x), out, g, row_bytes,
-                                                               h0 * d * esz, chunks, d);
+    summarize_kernel<false, MODE><<<(int)blocks, 256, 0, s>>>(a, b, out0, out1, g, row_bytes, h0 * d * esz, chunks, d);
   return cudaGetLastError();
 }
 
 cudaError_t launch_summarize(const void* x, float* out, const Geo& g, int heads_total, int h0, int hc, int d,
                              spade_dtype dt, int mode, cudaStream_t s) {
-  if (mode == 1) return launch_summarize_m<1>(x, out, g, heads_total, h0, hc, d, dt, s);
-  if (mode == 2) return launch_summarize_m<2>(x, out, g, heads_total, h0, hc, d, dt, s);
-  return launch_summarize_m<0>(x, out, g, heads_total, h0, hc, d, dt, s);
+  if (mode == 1) return launch_summarize_m<1>(x, nullptr, out, nullptr, g, heads_total, h0, hc, d, dt, s);
+  if (mode == 2) return launch_summarize_m<2>(x, nullptr, out, nullptr, g, heads_total, h0, hc, d, dt, s);
+  return launch_summarize_m<0>(x, nullptr, out, nullptr, g, heads_total, h0, hc, d, dt, s);
+}
+
+cudaError_t launch_summarize_pair(const void* q, const void* k, float* qout, float* kout, const Geo& g,
+                                  int heads_total, int h0, int hc, int d, spade_dtype dt, int mode, cudaStream_t s) {
+  if (mode == 1) return launch_summarize_m<1>(q, k, qout, kout, g, heads_total, h0, hc, d, dt, s);
+  if (mode == 2) return launch_summarize_m<2>(q, k, qout, kout, g, heads_total, h0, hc, d, dt, s);
+  return launch_summarize_m<0>(q, k, qout, kout, g, heads_total, h0, hc, d, dt, s);
 }
 
 }  // namespace spade

@@ -147,13 +147,18 @@ spade_status plan_group(const spade_geom* schemes, int n_schemes, const spade_he
 }
 
 // Step 3: the tensor-core estimator (split-precision TF32); the FMA-pipe
-// kernel only when the tensor-map encoder is unavailable.
-cudaError_t run_estimate(const float* qm, const float* km, float* prob, int heads, int nb, int d, int* status,
-                         cudaStream_t s) {
-  cudaError_t e = launch_estimate_tc(qm, km, prob, heads, nb, d, status, s);
+// kernel only when the tensor-map encoder is unavailable.  want_probs = false
+// asks for the scaled pooled scores (the index search then forms the
+// softmax); *holds_scores says which of the two `out` received (the FMA-pipe
+// kernel always writes probabilities).
+cudaError_t run_estimate(const float* qm, const float* km, float* out, int heads, int nb, int d, int* status,
+                         bool want_probs, bool* holds_scores, cudaStream_t s) {
+  cudaError_t e = launch_estimate_tc(qm, km, out, heads, nb, d, status, want_probs, s);
+  *holds_scores = !want_probs;
   if (e == cudaErrorNotSupported) {
     cudaGetLastError();
-    e = launch_estimate(qm, km, prob, heads, nb, d, s);
+    e = launch_estimate(qm, km, out, heads, nb, d, s);
+    *holds_scores = false;
   }
   return e;
 }
@@ -284,31 +289,81 @@ spade_status spade_summarize_mode(const void* x, float* out, spade_geom g, int h
   return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "summarize");
 }
 
-spade_status spade_estimate(const float* qmean, const float* kmean, float* prob, int heads, int nb, int d,
-                            spade_stream_t stream) {
-  if (!qmean || !kmean || !prob) return fail(SPADE_ERR_INVALID, "null pointer");
-  if (!aligned16(qmean) || !aligned16(kmean) || !aligned16(prob))
+spade_status spade_summarize_qk(const void* q, const void* k, float* qmean, float* kmean, spade_geom g, int heads,
+                                int d, spade_dtype dt, spade_stream_t stream) {
+  spade_status st = check_geom(g);
+  if (st != SPADE_OK) return st;
+  if ((st = check_d_dt(d, dt)) != SPADE_OK) return st;
+  if (!q || !k || !qmean || !kmean) return fail(SPADE_ERR_INVALID, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(qmean) || !aligned16(kmean))
+    return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  if (heads < 1) return fail(SPADE_ERR_INVALID, "heads=%d", heads);
+  cudaError_t e = launch_summarize_pair(q, k, qmean, kmean, make_geo(g), heads, 0, heads, d, dt, 0, as_cuda(stream));
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "summarize");
+}
+
+static spade_status check_estimate_args(const float* qmean, const float* kmean, const float* out, int heads, int nb,
+                                       int d) {
+  if (!qmean || !kmean || !out) return fail(SPADE_ERR_INVALID, "null pointer");
+  if (!aligned16(qmean) || !aligned16(kmean) || !aligned16(out))
     return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
   if (heads < 1 || heads > 65535) return fail(SPADE_ERR_INVALID, "heads=%d", heads);
   if (nb < 1) return fail(SPADE_ERR_INVALID, "nb=%d", nb);
   if (nb > SPADE_ESTIMATE_MAX_NB) return fail(SPADE_ERR_UNSUPPORTED, "nb=%d above %d", nb, SPADE_ESTIMATE_MAX_NB);
   if (d != 64 && d != 128) return fail(SPADE_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", d);
+  return SPADE_OK;
+}
+
+spade_status spade_estimate(const float* qmean, const float* kmean, float* prob, int heads, int nb, int d,
+                            spade_stream_t stream) {
+  spade_status st0 = check_estimate_args(qmean, kmean, prob, heads, nb, d);
+  if (st0 != SPADE_OK) return st0;
   int* st = status_ptr();
   if (!st) return fail(SPADE_ERR_CUDA, "device status word unavailable");
-  cudaError_t e = run_estimate(qmean, kmean, prob, heads, nb, d, st, as_cuda(stream));
+  bool scores = false;
+  cudaError_t e = run_estimate(qmean, kmean, prob, heads, nb, d, st, true, &scores, as_cuda(stream));
   return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "estimate");
 }
 
-spade_status spade_select(const float* prob, const float* tau_host, int* cnt, int* idx, int heads, int nb,
-                          spade_stream_t stream) {
-  if (!prob || !tau_host || !cnt || !idx) return fail(SPADE_ERR_INVALID, "null pointer");
+spade_status spade_estimate_scores(const float* qmean, const float* kmean, float* scores, int heads, int nb, int d,
+                                   spade_stream_t stream) {
+  spade_status st0 = check_estimate_args(qmean, kmean, scores, heads, nb, d);
+  if (st0 != SPADE_OK) return st0;
+  int* st = status_ptr();
+  if (!st) return fail(SPADE_ERR_CUDA, "device status word unavailable");
+  cudaError_t e = launch_estimate_tc(qmean, kmean, scores, heads, nb, d, st, false, as_cuda(stream));
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    return fail(SPADE_ERR_UNSUPPORTED, "tensor-map encoder unavailable: no score-only estimator");
+  }
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "estimate scores");
+}
+
+static spade_status check_select_args(const float* in, const float* tau_host, const int* cnt, const int* idx,
+                                     int heads, int nb) {
+  if (!in || !tau_host || !cnt || !idx) return fail(SPADE_ERR_INVALID, "null pointer");
   if (heads < 1 || heads > SPADE_SELECT_MAX_HEADS) return fail(SPADE_ERR_UNSUPPORTED, "heads=%d (1..1024)", heads);
   if (nb < 1) return fail(SPADE_ERR_INVALID, "nb=%d", nb);
   if (nb > SPADE_SELECT_MAX_NB) return fail(SPADE_ERR_UNSUPPORTED, "nb=%d above %d", nb, SPADE_SELECT_MAX_NB);
   for (int h = 0; h < heads; ++h)
     if (!(tau_host[h] > 0.f && tau_host[h] <= 1e30f)) return fail(SPADE_ERR_INVALID, "tau[%d] must be > 0", h);
+  return SPADE_OK;
+}
+
+spade_status spade_select(const float* prob, const float* tau_host, int* cnt, int* idx, int heads, int nb,
+                          spade_stream_t stream) {
+  spade_status st = check_select_args(prob, tau_host, cnt, idx, heads, nb);
+  if (st != SPADE_OK) return st;
   cudaError_t e = launch_select(prob, tau_host, cnt, idx, heads, nb, as_cuda(stream));
   return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "select");
+}
+
+spade_status spade_select_scores(const float* scores, const float* tau_host, int* cnt, int* idx, int heads, int nb,
+                                 spade_stream_t stream) {
+  spade_status st = check_select_args(scores, tau_host, cnt, idx, heads, nb);
+  if (st != SPADE_OK) return st;
+  cudaError_t e = launch_select(scores, tau_host, cnt, idx, heads, nb, as_cuda(stream), nullptr, nullptr, true);
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "select scores");
 }
 
 spade_status spade_select_window(const float* prob, const float* tau_host, const int* radius_host, spade_geom g,
@@ -524,15 +579,21 @@ spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, 
       int j = i + 1;
       while (j < hs && hl[j] == hl[j - 1] + 1) ++j;
       const size_t o = (size_t)i * g.nb * d;
-      cudaError_t e = launch_summarize(q, qm + o, g, heads, hl[i], j - i, d, dt, (int)q_summary, s);
-      if (e == cudaSuccess) e = launch_summarize(k, km + o, g, heads, hl[i], j - i, d, dt, (int)k_summary, s);
+      cudaError_t e;
+      if (q_summary == k_summary) {               // Q and K in one launch
+        e = launch_summarize_pair(q, k, qm + o, km + o, g, heads, hl[i], j - i, d, dt, (int)q_summary, s);
+      } else {
+        e = launch_summarize(q, qm + o, g, heads, hl[i], j - i, d, dt, (int)q_summary, s);
+        if (e == cudaSuccess) e = launch_summarize(k, km + o, g, heads, hl[i], j - i, d, dt, (int)k_summary, s);
+      }
       if (e != cudaSuccess) return cuda_fail(e, "summarize");
       i = j;
     }
     float* prob = reinterpret_cast<float*>(ws + L.prob[sc]);
     int* st = status_ptr();
     if (!st) return fail(SPADE_ERR_CUDA, "device status word unavailable");
-    cudaError_t e = run_estimate(qm, km, prob, hs, g.nb, d, st, s);
+    bool scores = false;
+    cudaError_t e = run_estimate(qm, km, prob, hs, g.nb, d, st, false, &scores, s);
     if (e != cudaSuccess) return cuda_fail(e, "estimate");
     std::vector<float> taus(hs);
     std::vector<int> rad(3 * hs, 0);
@@ -543,7 +604,7 @@ spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, 
     }
     e = launch_select(prob, taus.data(), reinterpret_cast<int*>(ws + L.cnt[sc]),
                       reinterpret_cast<int*>(ws + L.idx[sc]), hs, g.nb, s, window_radius ? rad.data() : nullptr,
-                      &g);
+                      &g, scores);
     if (e != cudaSuccess) return cuda_fail(e, "select");
   }
   // step 5: one grouped launch over every head

@@ -81,12 +81,19 @@ cudaError_t launch_tile3d(const void* x, void* xt, const Geo& g, int heads, int 
                           cudaStream_t s);
 cudaError_t launch_summarize(const void* x, float* out, const Geo& g, int heads_total, int h0, int hc, int d,
                              spade_dtype dt, int mode, cudaStream_t s);
-cudaError_t launch_estimate_tc(const float* qm, const float* km, float* prob, int heads, int nb, int d, int* status,
-                               cudaStream_t s);
+// Q and K with the same reduce, in one launch.
+cudaError_t launch_summarize_pair(const void* q, const void* k, float* qout, float* kout, const Geo& g,
+                                  int heads_total, int h0, int hc, int d, spade_dtype dt, int mode, cudaStream_t s);
+// probs = false: out = the scaled pooled scores; true: their row softmax.
+cudaError_t launch_estimate_tc(const float* qm, const float* km, float* out, int heads, int nb, int d, int* status,
+                               bool probs, cudaStream_t s);
 cudaError_t launch_estimate(const float* qm, const float* km, float* prob, int heads, int nb, int d,
                             cudaStream_t s);
-cudaError_t launch_select(const float* prob, const float* tau_host, int* cnt, int* idx, int heads, int nb,
-                          cudaStream_t s, const int* radius_host = nullptr, const Geo* g = nullptr);
+// scores = true: `in` holds scaled pooled scores and the kernel forms the
+// softmax itself; false: `in` holds probabilities.
+cudaError_t launch_select(const float* in, const float* tau_host, int* cnt, int* idx, int heads, int nb,
+                          cudaStream_t s, const int* radius_host = nullptr, const Geo* g = nullptr,
+                          bool scores = false);
 cudaError_t launch_worklist(const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 // Returns cudaErrorNotSupported if the shape is not for the tensor-core path.

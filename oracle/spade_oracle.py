@@ -48,7 +48,7 @@ from typing import Dict, List, Optional, Sequence, Tuple
 import numpy as np
 
 __all__ = [
-    "block_tokens", "valid_counts", "tile3d", "untile3d", "summarize", "estimate",
+    "block_tokens", "valid_counts", "tile3d", "untile3d", "summarize", "pooled_scores", "estimate", "softmax_rows",
     "select_row", "select", "selection_margin", "window_blocks", "attention_rows", "block_sparse_attention",
     "dense_attention", "pipeline", "kept_token_pairs",
     "block_sics", "sics", "choose_schemes",
@@ -143,10 +143,21 @@ def summarize(x: np.ndarray, geom: Sequence[int], mode: str = "mean") -> np.ndar
 # 3. Estimator: softmax over key blocks of pooled scores
 # ---------------------------------------------------------------------------
 
+def pooled_scores(qmean: np.ndarray, kmean: np.ndarray) -> np.ndarray:
+    """S[h, i, j] = Qbar[h,i] . Kbar[h,j] / sqrt(d): the Estimator's
+    inter-block score before its softmax."""
+    d = qmean.shape[-1]
+    return np.einsum("hid,hjd->hij", qmean.astype(np.float64), kmean.astype(np.float64)) / math.sqrt(d)
+
+
 def estimate(qmean: np.ndarray, kmean: np.ndarray) -> np.ndarray:
     """P[h, i, j] = softmax_j(Qbar[h,i] . Kbar[h,j] / sqrt(d))."""
-    d = qmean.shape[-1]
-    s = np.einsum("hid,hjd->hij", qmean.astype(np.float64), kmean.astype(np.float64)) / math.sqrt(d)
+    return softmax_rows(pooled_scores(qmean, kmean))
+
+
+def softmax_rows(s: np.ndarray) -> np.ndarray:
+    """softmax over the last axis, float64."""
+    s = np.asarray(s, dtype=np.float64)
     s = s - s.max(axis=-1, keepdims=True)
     e = np.exp(s)
     return e / e.sum(axis=-1, keepdims=True)

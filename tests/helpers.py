@@ -18,6 +18,7 @@ ATTN_MEAN_ABS_BF16 = 2e-3
 ATTN_MAX_ABS_F32 = 1e-4
 MEAN_REL = 1e-5
 PROB_ABS = 1e-5
+SCORE_REL = 2e-5      # pooled scores (split-precision TF32), relative to the largest |score|
 MARGIN = 1e-3
 
 

@@ -1,6 +1,8 @@
 """GPU parity, stage by stage, through the C ABI: tiling (bit-exact), block
 means (rel 1e-5), estimator probabilities (abs 1e-5), index search (bit-exact
 on rows whose oracle margin exceeds 1e-3), plus the bounded-wait error path."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -9,7 +11,7 @@ import oracle as O
 from input_adaptive_block_b200 import api
 from spade_workloads import Scheme, Workload, get_config, make_qkv
 
-from helpers import MARGIN, MEAN_REL, PROB_ABS, compare_kept, to_np
+from helpers import MARGIN, MEAN_REL, PROB_ABS, SCORE_REL, compare_kept, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +50,20 @@ def test_summarize(wl):
 
 
 @pytest.mark.parametrize("wl", RAGGED + [get_config("wan1.3b")], ids=lambda w: w.name)
+def test_summarize_qk(wl):
+    """Q and K in one launch: against the oracle, and bit-identical to the
+    one-tensor call (same per-unit arithmetic)."""
+    q, k, _ = make_qkv(wl, device="cuda")
+    geom = wl.schemes[0].as_tuple()
+    qm, km = api.summarize_qk(q, k, geom)
+    for x, got in ((q, qm), (k, km)):
+        ref = O.summarize(to_np(x[: wl.N]), geom)
+        err = np.abs(to_np(got) - ref) / np.maximum(np.abs(ref), 1.0)
+        assert err.max() <= MEAN_REL, err.max()
+        assert torch.equal(got, api.summarize(x, geom))
+
+
+@pytest.mark.parametrize("wl", RAGGED + [get_config("wan1.3b")], ids=lambda w: w.name)
 def test_estimate(wl):
     q, k, _ = make_qkv(wl, device="cuda")
     geom = wl.schemes[0].as_tuple()
@@ -66,6 +82,52 @@ def test_estimate_random_many_blocks():
     P = api.estimate(qm, km)
     ref = O.estimate(to_np(qm), to_np(km))
     assert np.abs(to_np(P) - ref).max() <= PROB_ABS
+
+
+@pytest.mark.parametrize("wl", RAGGED + [get_config("wan1.3b")], ids=lambda w: w.name)
+def test_estimate_scores(wl):
+    """The scores the grouped path hands to the fused softmax + index search."""
+    q, k, _ = make_qkv(wl, device="cuda")
+    geom = wl.schemes[0].as_tuple()
+    qm, km = api.summarize(q, geom), api.summarize(k, geom)
+    S = to_np(api.estimate_scores(qm, km))
+    ref = O.pooled_scores(to_np(qm), to_np(km))
+    assert S.shape == ref.shape
+    assert np.abs(S - ref).max() <= SCORE_REL * max(1.0, np.abs(ref).max())
+
+
+def test_estimate_scores_random_many_blocks():
+    """nb spanning several 128-block tiles with a ragged tail (1001 = 7 x 128 + 105,
+    so the last key tile runs a short MMA), d = 64 and 128."""
+    g = torch.Generator(device="cpu").manual_seed(12)
+    for d in (64, 128):
+        qm = (torch.randn(3, 1001, d, generator=g) * 0.6).cuda()
+        km = (torch.randn(3, 1001, d, generator=g) * 0.6).cuda()
+        S = to_np(api.estimate_scores(qm, km))
+        ref = O.pooled_scores(to_np(qm), to_np(km))
+        assert np.abs(S - ref).max() <= SCORE_REL * max(1.0, np.abs(ref).max()), d
+
+
+@pytest.mark.parametrize("wl", RAGGED + [get_config("wan1.3b")], ids=lambda w: w.name)
+def test_select_scores_against_oracle_chain(wl):
+    """The grouped path's steps 3-4 (scores, then the softmax fused into the
+    index search) against the oracle's fp64 chain."""
+    q, k, _ = make_qkv(wl, device="cuda")
+    geom = wl.schemes[0].as_tuple()
+    S = api.estimate_scores(api.summarize(q, geom), api.summarize(k, geom))
+    cnt, idx = api.select_scores(S, wl.head_tau)
+    cnt, idx = cnt.cpu().numpy(), idx.cpu().numpy()
+    Pref = O.estimate(O.summarize(to_np(q[: wl.N]), geom), O.summarize(to_np(k[: wl.N]), geom))
+    total_checked = 0
+    for h in range(wl.heads):
+        nb = Pref.shape[1]
+        gk = [list(idx[h, i, : cnt[h, i]]) for i in range(nb)]
+        ok = [O.select_row(Pref[h, i], i, wl.head_tau[h]) for i in range(nb)]
+        mg = [O.selection_margin(Pref[h, i], i, wl.head_tau[h]) for i in range(nb)]
+        checked, bad, _ = compare_kept(gk, ok, mg, P=Pref[h], tau=wl.head_tau[h])
+        assert not bad, (h, bad[:5])
+        total_checked += checked
+    assert total_checked >= 0.5 * wl.heads * Pref.shape[1]
 
 
 @pytest.mark.parametrize("wl", RAGGED + [get_config("wan1.3b")], ids=lambda w: w.name)
@@ -90,18 +152,28 @@ def test_select_against_oracle_chain(wl):
     assert total_checked >= 0.5 * wl.heads * Pref.shape[1]
 
 
-@pytest.mark.parametrize("nb", [5, 33, 100, 660, 1020, 1024])
-@pytest.mark.parametrize("tau", [0.3, 0.8, 0.9, 0.95, 0.999, 1.0])
-def test_select_random_rows(nb, tau):
-    """Synthetic probability rows with peaked and flat regions, exact ties
-    (uniform rows) and tau = 1; the oracle runs on the same fp32 values."""
+_ROWS = ([(nb, tau, "prob") for nb in (5, 33, 100, 630, 660, 1020, 1024) for tau in (0.3, 0.8, 0.9, 0.95, 0.999, 1.0)]
+         + [(nb, tau, "scores") for nb in (5, 33, 630, 1024) for tau in (0.3, 0.9, 0.999, 1.0)])
+
+
+@pytest.mark.parametrize("nb,tau,mode", _ROWS)
+def test_select_random_rows(nb, tau, mode):
+    """Synthetic rows with peaked and flat regions, exact ties (uniform rows)
+    and tau = 1, given as probabilities (the oracle runs on the same fp32
+    values) or as scores (the oracle runs on their fp64 softmax); nb = 630 is
+    a row length that is not a multiple of 4 (unaligned rows)."""
     g = torch.Generator(device="cpu").manual_seed(nb * 7 + int(tau * 1000))
     heads = 3
     logits = torch.randn(heads, nb, nb, generator=g, dtype=torch.float64) * torch.tensor([0.5, 2.0, 0.0]).view(3, 1, 1).double()
-    P = torch.softmax(logits, dim=-1).float()
-    cnt, idx = api.select(P.cuda(), [tau] * heads)
+    if mode == "prob":
+        P = torch.softmax(logits, dim=-1).float()
+        cnt, idx = api.select(P.cuda(), [tau] * heads)
+        Pn = P.double().numpy()
+    else:
+        S = logits.float()
+        cnt, idx = api.select_scores(S.cuda(), [tau] * heads)
+        Pn = O.softmax_rows(S.double().numpy())
     cnt, idx = cnt.cpu().numpy(), idx.cpu().numpy()
-    Pn = P.double().numpy()
     for h in range(heads):
         gk = [list(idx[h, i, : cnt[h, i]]) for i in range(nb)]
         ok = [O.select_row(Pn[h, i], i, tau) for i in range(nb)]

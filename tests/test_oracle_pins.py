@@ -108,6 +108,24 @@ def test_estimate_closed_forms():
     assert P[0, 1] == pytest.approx([0.5, 0.5], abs=1e-15)
 
 
+def test_pooled_scores_hand_worked():
+    # d = 4, sqrt(d) = 2.  Q rows (1,2,0,0), (0,0,1,1); K rows (1,0,0,0), (0,1,1,0):
+    # q0.k0 = 1, q0.k1 = 2, q1.k0 = 0, q1.k1 = 1  ->  S = [[0.5, 1.0], [0.0, 0.5]]
+    qm = np.array([[[1, 2, 0, 0], [0, 0, 1, 1]]], dtype=np.float64)
+    km = np.array([[[1, 0, 0, 0], [0, 1, 1, 0]]], dtype=np.float64)
+    S = O.pooled_scores(qm, km)
+    assert S.shape == (1, 2, 2)
+    assert np.array_equal(S[0], np.array([[0.5, 1.0], [0.0, 0.5]]))
+    # two heads are independent: the second head's scores do not mix with the first's
+    qm2 = np.concatenate([qm, 3 * qm])
+    km2 = np.concatenate([km, km])
+    assert np.array_equal(O.pooled_scores(qm2, km2)[1], 3 * S[0])
+    # the estimator is exactly the row softmax of these scores: S row 0 -> [e^0.5, e^1] / sum
+    P = O.estimate(qm, km)
+    e0, e1 = math.exp(0.5), math.exp(1.0)
+    assert P[0, 0] == pytest.approx([e0 / (e0 + e1), e1 / (e0 + e1)], abs=1e-15)
+
+
 def test_estimate_rows_sum_to_one_and_uniform_rank1():
     rng = np.random.default_rng(3)
     P = O.estimate(rng.standard_normal((3, 17, 64)) * 4, rng.standard_normal((3, 17, 64)) * 4)
