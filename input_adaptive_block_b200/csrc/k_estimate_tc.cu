@@ -13,16 +13,23 @@
 // (exact in fp32), and S = Qhi Khi^T + Qhi Klo^T + Qlo Khi^T (the lo lo term
 // and the TF32 rounding of lo are below 2^-20 relative).
 //
-//  * Persistent CTAs over items (head, 128 query rows, 128 key columns),
-//    dealt round-robin, so the work is spread evenly over the SMs.  Per item
-//    and 32-element d chunk: TMA loads the fp32 Q and K chunks (128 rows x
-//    128 B, 128-byte swizzled: the K-major layout the MMA reads); a converter
-//    warpgroup rewrites each chunk as hi in place and lo beside it (the split
-//    is elementwise, so the swizzled layout carries over); one thread issues
-//    the 12 tcgen05.mma (kind::tf32, M=128, K=8, N = the item's valid key
-//    columns rounded up to 16) into one of two S tiles in TMEM.
+//  * Persistent CTAs, each over a contiguous range of items (head, 128 query
+//    rows, 128 key columns), so the query tile changes only a few times per
+//    CTA.  The query tile lives in TMEM: a converter warpgroup (thread =
+//    query row) reads it from global memory, splits it and writes Qhi and
+//    Qlo with tcgen05.st; the MMAs read them as the A operand, so only key
+//    chunks pass through shared memory.  Per item and 32-element d chunk:
+//    TMA loads the fp32 K chunk (128 rows x 128 B, 128-byte swizzled: the
+//    K-major layout the MMA reads) into one of six stages; the converter
+//    rewrites it as hi in place and lo beside it (elementwise, so the
+//    swizzled layout carries over); one thread issues the 12 tcgen05.mma
+//    (kind::tf32, M=128, K=8, N = the item's valid key columns rounded up to
+//    16) into one of two S tiles in TMEM.
 //  * Two epilogue warpgroups (64 columns each; thread = query row) read a
-//    finished tile with tcgen05.ld, release it, scale it and store it.
+//    finished tile with tcgen05.ld, release it, scale it into a 128-byte
+//    swizzled shared-memory stage (one per warp) and write it with TMA
+//    tensor stores, whole 128-byte lines (a row per thread would touch 32
+//    lines per store instruction).
 //  * Every wait is bounded (globaltimer); a timeout latches SPADE_ERR_TIMEOUT
 //    in the device status word and the CTA winds down.
 #include <cudaTypedefs.h>
@@ -33,16 +40,22 @@
 namespace spade {
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kStages = 5;
 constexpr int kChunk = 128 * 128;           // 128 rows x 128 B (32 fp32 of d)
-constexpr int kStageBytes = 4 * kChunk;     // Q hi, Q lo, K hi, K lo
+constexpr int kStageBytes = 2 * kChunk;     // K hi (written over the landed chunk), K lo
 constexpr int kThreads = 512;               // producer, MMA, 2 idle, converters (4 warps), 2 x epilogue (4 warps)
-constexpr int kSmem = kStages * kStageBytes + 256 + 1024;
+constexpr int kOutBox = 32 * 128;           // one 32-row x 32-column fp32 box of scores, 128-byte swizzled
+constexpr int kOutWarpBytes = 2 * kOutBox;  // an epilogue warp's 64 columns of its 32 rows
+constexpr int kSmem = kStages * kStageBytes + 8 * kOutWarpBytes + 256 + 1024;
+// TMEM columns: S tiles [0, 256), Qhi [256, 256 + d), Qlo [384, 384 + d)
+constexpr uint32_t kColQhi = 256, kColQlo = 384;
 
 struct __align__(64) EstTcParams {
-  CUtensorMap tm_q, tm_k;   // [heads][nb][d] fp32: dims {d, nb, heads}, box {32, 128, 1}
+  CUtensorMap tm_k;         // [heads][nb][d] fp32: dims {d, nb, heads}, box {32, 128, 1}
+  CUtensorMap tm_out;       // [heads][nb][nb] fp32: dims {nb, nb, heads}, box {32, 32, 1} (OUT_TMA only)
+  const float* qm;          // [heads][nb][d] fp32
   float* out;               // [heads][nb][nb] scores
-  int nb, d, nrt, n_items;
+  int nb, d, nt, n_items;
   float scale;
   int* status;
   long long timeout_ns;
@@ -84,16 +97,28 @@ __device__ __forceinline__ uint32_t idesc_tf32(uint32_t n) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
+__device__ __forceinline__ uint32_t tf32_hi(uint32_t x) { return x & 0xFFFFE000u; }
+__device__ __forceinline__ uint32_t tf32_lo(uint32_t x) {
+  return __float_as_uint(__uint_as_float(x) - __uint_as_float(tf32_hi(x)));
+}
+
+// OUT_TMA: scores leave through a shared-memory stage and TMA tensor stores
+// (whole 128-byte lines; the tensor map clips rows and columns past nb);
+// otherwise (rows not 16-byte aligned: nb % 4 != 0) each thread stores its row.
+template <bool OUT_TMA>
 __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_constant__ EstTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* out_stage = smem + kStages * kStageBytes;   // 1024-byte aligned: 8 warps x kOutWarpBytes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + 8 * kOutWarpBytes);
   uint64_t* full = bars;                   // [kStages] TMA landed
   uint64_t* conv = bars + kStages;         // [kStages] split into hi / lo (128 threads)
   uint64_t* empty = bars + 2 * kStages;    // [kStages] MMAs done with the stage
   uint64_t* s_full = bars + 3 * kStages;   // [2] S tile complete
   uint64_t* s_free = s_full + 2;           // [2] S tile read (256 epilogue threads)
-  uint64_t* fin = s_full + 4;
+  uint64_t* q_full = s_full + 4;           // query tile in TMEM (128 threads)
+  uint64_t* q_free = s_full + 5;           // MMAs of the previous query tile done
+  uint64_t* fin = s_full + 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -108,16 +133,18 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
       ptx::mbar_init(&s_full[b], 1);
       ptx::mbar_init(&s_free[b], 256);
     }
+    ptx::mbar_init(q_full, 128);
+    ptx::mbar_init(q_free, 1);
     ptx::mbar_init(fin, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    ptx::prefetch_tmap(&p.tm_q);
     ptx::prefetch_tmap(&p.tm_k);
+    if (OUT_TMA) ptx::prefetch_tmap(&p.tm_out);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_slot, 256);
+    ptx::tmem_alloc(tmem_slot, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -125,24 +152,24 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const EWaiter W{abort_flag, p.status, p.timeout_ns};
-  const int nt = p.nrt;           // key tiles = query tiles (both cover nb in 128s)
+  const int nt = p.nt;            // key tiles = query tiles (both cover nb in 128s)
   const int ndc = p.d / 32;
+  // this CTA's items: a contiguous range of the (head, query tile, key tile) order
+  const int it0 = (int)((long long)blockIdx.x * p.n_items / gridDim.x);
+  const int it1 = (int)((long long)(blockIdx.x + 1) * p.n_items / gridDim.x);
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     uint32_t g = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
-      const int h = it / (nt * nt), rem = it - h * nt * nt;
-      const int rt = rem / nt, ct = rem - rt * nt;
+    for (int it = it0; ok && it < it1; ++it) {
+      const int h = it / (nt * nt), ct = it % nt;
       for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
         const int s = (int)(g % kStages);
         ok = __all_sync(0xffffffffu, ewait(&empty[s], ((g / kStages) & 1) ^ 1, W));
         if (!ok) break;
-        uint8_t* st = smem + s * kStageBytes;
-        ptx::mbar_arrive_expect_tx_elect(&full[s], 2 * kChunk);
-        ptx::tma_load_3d_elect(st, &p.tm_q, &full[s], 32 * dc, 128 * rt, h);
-        ptx::tma_load_3d_elect(st + 2 * kChunk, &p.tm_k, &full[s], 32 * dc, 128 * ct, h);
+        ptx::mbar_arrive_expect_tx_elect(&full[s], kChunk);
+        ptx::tma_load_3d_elect(smem + s * kStageBytes, &p.tm_k, &full[s], 32 * dc, 128 * ct, h);
       }
     }
     if (lane == 0 && !ok && g > 0) {   // wind down: let the loads issued land
@@ -151,15 +178,23 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer --
-    uint32_t g = 0, gi = 0;
+    uint32_t g = 0, gi = 0, gq = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++gi) {
-      const int ct = (it % (nt * nt)) % nt;
+    for (int it = it0; ok && it < it1; ++it, ++gi) {
+      if (it == it0 || it % nt == 0) {                 // a new query tile
+        if (gq > 0) ptx::tc_commit_elect(q_free);      // fires once the previous tile's MMAs are done
+        ok = __all_sync(0xffffffffu, ewait(q_full, gq & 1, W));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        ++gq;
+      }
+      const int ct = it % nt;
       const int nv = p.nb - 128 * ct < 128 ? p.nb - 128 * ct : 128;   // valid key columns
       const uint32_t idesc = idesc_tf32((uint32_t)((nv + 15) & ~15));
       const int b = (int)(gi & 1);
       ok = __all_sync(0xffffffffu, ewait(&s_free[b], ((gi >> 1) & 1) ^ 1, W));
       if (!ok) break;
+      ptx::tc_fence_after();
       const uint32_t ts = tmem + 128 * b;
       for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
         const int s = (int)(g % kStages);
@@ -167,14 +202,14 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
         if (!ok) break;
         ptx::tc_fence_after();
         const uint32_t base = ptx::smem_u32(smem + s * kStageBytes);
-        const uint64_t qhi = kdesc(base), qlo = kdesc(base + kChunk);
-        const uint64_t khi = kdesc(base + 2 * kChunk), klo = kdesc(base + 3 * kChunk);
+        const uint64_t khi = kdesc(base), klo = kdesc(base + kChunk);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {           // 8 fp32 (32 B) of d per MMA
           const uint64_t off = (uint64_t)((kk * 32) >> 4);
-          ptx::mma_ss_tf32_elect(ts, qhi + off, khi + off, idesc, (dc > 0 || kk > 0) ? 1u : 0u);
-          ptx::mma_ss_tf32_elect(ts, qhi + off, klo + off, idesc, 1u);
-          ptx::mma_ss_tf32_elect(ts, qlo + off, khi + off, idesc, 1u);
+          const uint32_t ac = (uint32_t)(32 * dc + 8 * kk);
+          ptx::mma_ts_tf32_elect(ts, tmem + kColQhi + ac, khi + off, idesc, (dc > 0 || kk > 0) ? 1u : 0u);
+          ptx::mma_ts_tf32_elect(ts, tmem + kColQhi + ac, klo + off, idesc, 1u);
+          ptx::mma_ts_tf32_elect(ts, tmem + kColQlo + ac, khi + off, idesc, 1u);
         }
         ptx::tc_commit_elect(&empty[s]);
       }
@@ -183,45 +218,70 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     ptx::tc_commit_elect(fin);
     edrain(fin, 0, 100000000LL);
   } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------- hi / lo converters --
+    // -------------------------- query tile into TMEM, K chunks into hi / lo --
     const int ctid = threadIdx.x - 128;
-    uint32_t g = 0;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    uint32_t g = 0, gq = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x)
-        for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
-          const int s = (int)(g % kStages);
-          ok = ewait(&full[s], (g / kStages) & 1, W);
+    for (int it = it0; ok && it < it1; ++it) {
+      if (it == it0 || it % nt == 0) {
+        if (gq > 0) {
+          ok = ewait(q_free, (gq - 1) & 1, W);         // the previous tile's MMAs have read it
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-          uint8_t* st = smem + s * kStageBytes;
-#pragma unroll 4
-          for (int i = ctid; i < 2 * (kChunk / 16); i += 128) {
-            const int region = i / (kChunk / 16);          // 0: Q, 1: K
-            uint4* hi = reinterpret_cast<uint4*>(st + region * 2 * kChunk) + (i % (kChunk / 16));
-            uint4* lo = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(hi) + kChunk);
-            const uint4 v = *hi;
-            const uint4 h4 = make_uint4(v.x & 0xFFFFE000u, v.y & 0xFFFFE000u, v.z & 0xFFFFE000u, v.w & 0xFFFFE000u);
-            const uint4 l4 = make_uint4(__float_as_uint(__uint_as_float(v.x) - __uint_as_float(h4.x)),
-                                        __float_as_uint(__uint_as_float(v.y) - __uint_as_float(h4.y)),
-                                        __float_as_uint(__uint_as_float(v.z) - __uint_as_float(h4.z)),
-                                        __float_as_uint(__uint_as_float(v.w) - __uint_as_float(h4.w)));
-            *hi = h4;
-            *lo = l4;
-          }
-          ptx::fence_proxy_async_smem();                   // generic writes -> tensor-core reads
-          ptx::mbar_arrive(&conv[s]);
+          ptx::tc_fence_after();
         }
+        const int h = it / (nt * nt), rt = (it / nt) % nt;
+        const int i = 128 * rt + row;
+        const float4* src = reinterpret_cast<const float4*>(p.qm + ((long long)h * p.nb + (i < p.nb ? i : 0)) * p.d);
+        for (int c0 = 0; c0 < p.d; c0 += 32) {
+          uint32_t hi[32], lo[32];
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < p.nb) v = __ldg(src + c0 / 4 + q4);
+            const uint32_t x[4] = {__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
+                                   __float_as_uint(v.w)};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              hi[4 * q4 + e] = tf32_hi(x[e]);
+              lo[4 * q4 + e] = tf32_lo(x[e]);
+            }
+          }
+          ptx::tmem_st32(tmem + lane_base + kColQhi + c0, hi);
+          ptx::tmem_st32(tmem + lane_base + kColQlo + c0, lo);
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(q_full);
+        ++gq;
+      }
+      for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
+        const int s = (int)(g % kStages);
+        ok = ewait(&full[s], (g / kStages) & 1, W);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        uint4* hi4 = reinterpret_cast<uint4*>(smem + s * kStageBytes);
+        uint4* lo4 = reinterpret_cast<uint4*>(smem + s * kStageBytes + kChunk);
+#pragma unroll 4
+        for (int q = ctid; q < kChunk / 16; q += 128) {
+          const uint4 v = hi4[q];
+          hi4[q] = make_uint4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+          lo4[q] = make_uint4(tf32_lo(v.x), tf32_lo(v.y), tf32_lo(v.z), tf32_lo(v.w));
+        }
+        ptx::fence_proxy_async_smem();                 // generic writes -> tensor-core reads
+        ptx::mbar_arrive(&conv[s]);
+      }
+    }
   } else if (warp >= 8) {
     // --------------------------------------------------------- epilogues --
     const int half = (warp - 8) >> 2;            // key columns 64*half .. 64*half + 63 of the tile
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    const bool vec = (p.nb & 3) == 0;
     uint32_t gi = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x, ++gi) {
-      const int h = it / (nt * nt), rem = it - h * nt * nt;
-      const int rt = rem / nt, ct = rem - rt * nt;
+    for (int it = it0; ok && it < it1; ++it, ++gi) {
+      const int h = it / (nt * nt), rt = (it / nt) % nt, ct = it % nt;
       const int b = (int)(gi & 1);
       ok = ewait(&s_full[b], (gi >> 1) & 1, W);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -233,27 +293,45 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
       if (nv > 0) ptx::tmem_ld64(tmem + lane_base + 128 * b + 64 * half, sr);
       ptx::tc_fence_before();
       ptx::mbar_arrive(&s_free[b]);                // the tile may be overwritten now
-      if (nv > 0 && i < p.nb) {
-        float* dst = p.out + ((long long)h * p.nb + i) * p.nb + j0;
-        if (vec) {
+      if (OUT_TMA) {
+        if (nv > 0) {
+          uint8_t* st = out_stage + (warp - 8) * kOutWarpBytes;
+          if (lane == 0) ptx::bulk_wait_read0();   // this warp's previous stores have read the stage
+          __syncwarp();
+          // row `lane` of the warp's 32-row boxes; 16-byte chunk c of the
+          // 128-byte box row sits at chunk position c ^ (row & 7)
 #pragma unroll
-          for (int c4 = 0; c4 < 16; ++c4)
-            if (4 * c4 < nv)
-              reinterpret_cast<float4*>(dst)[c4] =
-                  make_float4(__uint_as_float(sr[4 * c4]) * p.scale, __uint_as_float(sr[4 * c4 + 1]) * p.scale,
-                              __uint_as_float(sr[4 * c4 + 2]) * p.scale, __uint_as_float(sr[4 * c4 + 3]) * p.scale);
-        } else {
+          for (int q = 0; q < 2; ++q)
+            if (32 * q < nv) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < nv) dst[c] = __uint_as_float(sr[c]) * p.scale;
+              for (int c = 0; c < 8; ++c) {
+                const uint32_t* v = sr + 32 * q + 4 * c;
+                *reinterpret_cast<float4*>(st + q * kOutBox + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                    make_float4(__uint_as_float(v[0]) * p.scale, __uint_as_float(v[1]) * p.scale,
+                                __uint_as_float(v[2]) * p.scale, __uint_as_float(v[3]) * p.scale);
+              }
+            }
+          ptx::fence_proxy_async_smem();             // generic writes -> TMA reads
+          __syncwarp();
+          if (lane == 0) {
+            for (int q = 0; q < 2; ++q)
+              if (32 * q < nv) ptx::tma_store_3d(&p.tm_out, st + q * kOutBox, j0 + 32 * q, 128 * rt + 32 * quad, h);
+            ptx::bulk_commit();
+          }
         }
+      } else if (nv > 0 && i < p.nb) {
+        float* dst = p.out + ((long long)h * p.nb + i) * p.nb + j0;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c < nv) dst[c] = __uint_as_float(sr[c]) * p.scale;
       }
     }
+    if (OUT_TMA && lane == 0) ptx::bulk_wait0();     // stores complete before the CTA exits
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == 1) ptx::tmem_dealloc(tmem, 256);
+  if (warp == 1) ptx::tmem_dealloc(tmem, 512);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -317,30 +395,46 @@ cudaError_t launch_softmax_rows(float* s, long long rows, int nb, cudaStream_t s
   return cudaGetLastError();
 }
 
+bool map_scores(CUtensorMap* m, float* base, int heads, int nb) {
+  cuuint64_t dims[3] = {(cuuint64_t)nb, (cuuint64_t)nb, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)nb * 4, (cuuint64_t)nb * nb * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_estimate_tc(const float* qm, const float* km, float* out, int heads, int nb, int d, int* status,
                                bool probs, cudaStream_t s) {
   if (!encode_fn()) return cudaErrorNotSupported;
-  if (d % 32 != 0 || (reinterpret_cast<uintptr_t>(qm) & 15) || (reinterpret_cast<uintptr_t>(km) & 15))
+  if (d % 32 != 0 || d > 128 || (reinterpret_cast<uintptr_t>(qm) & 15) || (reinterpret_cast<uintptr_t>(km) & 15))
     return cudaErrorInvalidValue;
   static EstTcParams tp;
   memset(&tp, 0, sizeof(tp));
-  if (!map_means(&tp.tm_q, qm, heads, nb, d) || !map_means(&tp.tm_k, km, heads, nb, d)) return cudaErrorInvalidValue;
+  if (!map_means(&tp.tm_k, km, heads, nb, d)) return cudaErrorInvalidValue;
+  tp.qm = qm;
   tp.out = out;
   tp.nb = nb;
   tp.d = d;
-  tp.nrt = (nb + 127) / 128;
-  tp.n_items = heads * tp.nrt * tp.nrt;
+  tp.nt = (nb + 127) / 128;
+  tp.n_items = heads * tp.nt * tp.nt;
   tp.scale = 1.0f / sqrtf((float)d);
   tp.status = status;
   tp.timeout_ns = device_wait_timeout_ns();
   static_assert(kSmem <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(estimate_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  // TMA stores need 16-byte row strides and a 16-byte aligned base
+  const bool out_tma = nb % 4 == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0 &&
+                       map_scores(&tp.tm_out, out, heads, nb);
+  cudaError_t e = cudaFuncSetAttribute(out_tma ? estimate_tc_kernel<true> : estimate_tc_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   const int grid = tp.n_items < num_sms() ? tp.n_items : num_sms();
   if (grid <= 0) return cudaSuccess;
-  estimate_tc_kernel<<<grid, kThreads, kSmem, s>>>(tp);
+  if (out_tma) estimate_tc_kernel<true><<<grid, kThreads, kSmem, s>>>(tp);
+  else estimate_tc_kernel<false><<<grid, kThreads, kSmem, s>>>(tp);
   e = cudaGetLastError();
   if (e != cudaSuccess || !probs) return e;
   const long long rows = (long long)heads * nb;
