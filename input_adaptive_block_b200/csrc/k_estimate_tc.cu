@@ -16,7 +16,8 @@
 //  * Persistent CTAs, each over a contiguous range of items (head, 128 query
 //    rows, 128 key columns), so the query tile changes only a few times per
 //    CTA.  The query tile lives in TMEM: a converter warpgroup (thread =
-//    query row) reads it from global memory, splits it and writes Qhi and
+//    query row) reads it from global memory (the next 32 columns' loads in
+//    flight while the current ones are split), splits it and writes Qhi and
 //    Qlo with tcgen05.st; the MMAs read them as the A operand, so only key
 //    chunks pass through shared memory.  Per item and 32-element d chunk:
 //    TMA loads the fp32 K chunk (128 rows x 128 B, 128-byte swizzled: the
@@ -26,10 +27,11 @@
 //    (kind::tf32, M=128, K=8, N = the item's valid key columns rounded up to
 //    16) into one of two S tiles in TMEM.
 //  * Two epilogue warpgroups (64 columns each; thread = query row) read a
-//    finished tile with tcgen05.ld, release it, scale it into a 128-byte
-//    swizzled shared-memory stage (one per warp) and write it with TMA
-//    tensor stores, whole 128-byte lines (a row per thread would touch 32
-//    lines per store instruction).
+//    finished tile with tcgen05.ld, release it, scale it, transpose 8x8
+//    blocks of 16-byte chunks across each 8-lane group with shuffles, and
+//    store whole 128-byte row segments, four rows per store instruction
+//    (a row per thread would touch 32 lines per instruction; a shared-memory
+//    stage would compete with the MMA operands for shared-memory bandwidth).
 //  * Every wait is bounded (globaltimer); a timeout latches SPADE_ERR_TIMEOUT
 //    in the device status word and the CTA winds down.
 #include <cudaTypedefs.h>
@@ -40,19 +42,16 @@
 namespace spade {
 namespace {
 
-constexpr int kStages = 5;
+constexpr int kStages = 6;
 constexpr int kChunk = 128 * 128;           // 128 rows x 128 B (32 fp32 of d)
 constexpr int kStageBytes = 2 * kChunk;     // K hi (written over the landed chunk), K lo
 constexpr int kThreads = 512;               // producer, MMA, 2 idle, converters (4 warps), 2 x epilogue (4 warps)
-constexpr int kOutBox = 32 * 128;           // one 32-row x 32-column fp32 box of scores, 128-byte swizzled
-constexpr int kOutWarpBytes = 2 * kOutBox;  // an epilogue warp's 64 columns of its 32 rows
-constexpr int kSmem = kStages * kStageBytes + 8 * kOutWarpBytes + 256 + 1024;
+constexpr int kSmem = kStages * kStageBytes + 256 + 1024;
 // TMEM columns: S tiles [0, 256), Qhi [256, 256 + d), Qlo [384, 384 + d)
 constexpr uint32_t kColQhi = 256, kColQlo = 384;
 
 struct __align__(64) EstTcParams {
   CUtensorMap tm_k;         // [heads][nb][d] fp32: dims {d, nb, heads}, box {32, 128, 1}
-  CUtensorMap tm_out;       // [heads][nb][nb] fp32: dims {nb, nb, heads}, box {32, 32, 1} (OUT_TMA only)
   const float* qm;          // [heads][nb][d] fp32
   float* out;               // [heads][nb][nb] scores
   int nb, d, nt, n_items;
@@ -101,16 +100,73 @@ __device__ __forceinline__ uint32_t tf32_hi(uint32_t x) { return x & 0xFFFFE000u
 __device__ __forceinline__ uint32_t tf32_lo(uint32_t x) {
   return __float_as_uint(__uint_as_float(x) - __uint_as_float(tf32_hi(x)));
 }
+__device__ __forceinline__ uint32_t tf32_hi(float x) { return tf32_hi(__float_as_uint(x)); }
+__device__ __forceinline__ uint32_t tf32_lo(float x) { return tf32_lo(__float_as_uint(x)); }
 
-// OUT_TMA: scores leave through a shared-memory stage and TMA tensor stores
-// (whole 128-byte lines; the tensor map clips rows and columns past nb);
-// otherwise (rows not 16-byte aligned: nb % 4 != 0) each thread stores its row.
-template <bool OUT_TMA>
+__device__ __forceinline__ void load8(float4 (&v)[8], const float4* src, bool valid) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) v[q] = valid ? __ldg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// Rows 32*(warp&3) .. +31 of the query tile (head h, tile rt) into TMEM as
+// TF32 hi / lo: one row per thread, 32 columns per tcgen05.st, the next 32
+// columns' loads in flight while the current ones are split and stored.
+__device__ __forceinline__ void load_q_tile(const EstTcParams& p, int h, int rt, int quad, int lane, uint32_t tmem) {
+  const int i = 128 * rt + quad * 32 + lane;
+  const bool valid = i < p.nb;
+  const float4* src = reinterpret_cast<const float4*>(p.qm + ((long long)h * p.nb + (valid ? i : 0)) * p.d);
+  const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+  float4 cur[8], nxt[8];
+  load8(cur, src, valid);
+  for (int c0 = 0; c0 < p.d; c0 += 32) {
+    if (c0 + 32 < p.d) load8(nxt, src + (c0 + 32) / 4, valid);
+    uint32_t r[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      r[4 * q] = tf32_hi(cur[q].x); r[4 * q + 1] = tf32_hi(cur[q].y);
+      r[4 * q + 2] = tf32_hi(cur[q].z); r[4 * q + 3] = tf32_hi(cur[q].w);
+    }
+    ptx::tmem_st32(tmem + lane_base + kColQhi + c0, r);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      r[4 * q] = tf32_lo(cur[q].x); r[4 * q + 1] = tf32_lo(cur[q].y);
+      r[4 * q + 2] = tf32_lo(cur[q].z); r[4 * q + 3] = tf32_lo(cur[q].w);
+    }
+    ptx::tmem_st32(tmem + lane_base + kColQlo + c0, r);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) cur[q] = nxt[q];
+  }
+}
+
+__device__ __forceinline__ float4 shfl_xor4(float4 v, int m) {
+  return make_float4(__shfl_xor_sync(0xffffffffu, v.x, m), __shfl_xor_sync(0xffffffffu, v.y, m),
+                     __shfl_xor_sync(0xffffffffu, v.z, m), __shfl_xor_sync(0xffffffffu, v.w, m));
+}
+// 8x8 transpose of 16-byte elements across each 8-lane group: on entry lane
+// 8G + r holds e[k] = element (r, k); on exit lane 8G + k holds e[r] = (r, k).
+__device__ __forceinline__ void transpose8(float4 (&e)[8], int lane) {
+#pragma unroll
+  for (int s = 4; s >= 1; s >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j & s) continue;
+      const float4 send = upper ? e[j] : e[j | s];
+      const float4 recv = shfl_xor4(send, s);
+      if (upper) e[j] = recv; else e[j | s] = recv;
+    }
+  }
+}
+
+
+
+// VEC: nb % 4 == 0 (16-byte aligned score rows): transposed whole-line
+// stores; otherwise each thread stores its own row.
+template <bool VEC>
 __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_constant__ EstTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* out_stage = smem + kStages * kStageBytes;   // 1024-byte aligned: 8 warps x kOutWarpBytes
-  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + 8 * kOutWarpBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
   uint64_t* full = bars;                   // [kStages] TMA landed
   uint64_t* conv = bars + kStages;         // [kStages] split into hi / lo (128 threads)
   uint64_t* empty = bars + 2 * kStages;    // [kStages] MMAs done with the stage
@@ -139,10 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    ptx::prefetch_tmap(&p.tm_k);
-    if (OUT_TMA) ptx::prefetch_tmap(&p.tm_out);
-  }
+  if (warp == 0 && lane == 0) ptx::prefetch_tmap(&p.tm_k);
   if (warp == 1) {
     ptx::tmem_alloc(tmem_slot, 512);
     ptx::tmem_relinquish();
@@ -221,8 +274,6 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     // -------------------------- query tile into TMEM, K chunks into hi / lo --
     const int ctid = threadIdx.x - 128;
     const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     uint32_t g = 0, gq = 0;
     bool ok = true;
     for (int it = it0; ok && it < it1; ++it) {
@@ -232,26 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           ptx::tc_fence_after();
         }
-        const int h = it / (nt * nt), rt = (it / nt) % nt;
-        const int i = 128 * rt + row;
-        const float4* src = reinterpret_cast<const float4*>(p.qm + ((long long)h * p.nb + (i < p.nb ? i : 0)) * p.d);
-        for (int c0 = 0; c0 < p.d; c0 += 32) {
-          uint32_t hi[32], lo[32];
-#pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < p.nb) v = __ldg(src + c0 / 4 + q4);
-            const uint32_t x[4] = {__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
-                                   __float_as_uint(v.w)};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              hi[4 * q4 + e] = tf32_hi(x[e]);
-              lo[4 * q4 + e] = tf32_lo(x[e]);
-            }
-          }
-          ptx::tmem_st32(tmem + lane_base + kColQhi + c0, hi);
-          ptx::tmem_st32(tmem + lane_base + kColQlo + c0, lo);
-        }
+        load_q_tile(p, it / (nt * nt), (it / nt) % nt, quad, lane, tmem);
         ptx::tc_fence_before();
         ptx::mbar_arrive(q_full);
         ++gq;
@@ -276,7 +308,6 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     // --------------------------------------------------------- epilogues --
     const int half = (warp - 8) >> 2;            // key columns 64*half .. 64*half + 63 of the tile
     const int quad = warp & 3;
-    const int row = quad * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     uint32_t gi = 0;
     bool ok = true;
@@ -286,47 +317,46 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
       ok = ewait(&s_full[b], (gi >> 1) & 1, W);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       ptx::tc_fence_after();
-      const int i = 128 * rt + row;
       const int j0 = 128 * ct + 64 * half;
       const int nv = p.nb - j0 < 64 ? p.nb - j0 : 64;   // valid columns of this half (warp-uniform)
       uint32_t sr[64];
       if (nv > 0) ptx::tmem_ld64(tmem + lane_base + 128 * b + 64 * half, sr);
       ptx::tc_fence_before();
       ptx::mbar_arrive(&s_free[b]);                // the tile may be overwritten now
-      if (OUT_TMA) {
-        if (nv > 0) {
-          uint8_t* st = out_stage + (warp - 8) * kOutWarpBytes;
-          if (lane == 0) ptx::bulk_wait_read0();   // this warp's previous stores have read the stage
-          __syncwarp();
-          // row `lane` of the warp's 32-row boxes; 16-byte chunk c of the
-          // 128-byte box row sits at chunk position c ^ (row & 7)
+      if (nv <= 0) continue;
+      const int row0 = 128 * rt + 32 * quad;       // this warp's first query row
+      float* base = p.out + (long long)h * p.nb * p.nb;
+      if (VEC) {
+        const int grp = lane >> 3, k = lane & 7;
 #pragma unroll
-          for (int q = 0; q < 2; ++q)
-            if (32 * q < nv) {
+        for (int blk = 0; blk < 2; ++blk) {
+          float4 e[8];
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const uint32_t* v = sr + 32 * q + 4 * c;
-                *reinterpret_cast<float4*>(st + q * kOutBox + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                    make_float4(__uint_as_float(v[0]) * p.scale, __uint_as_float(v[1]) * p.scale,
-                                __uint_as_float(v[2]) * p.scale, __uint_as_float(v[3]) * p.scale);
-              }
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t* v = sr + 32 * blk + 4 * c;
+            e[c] = make_float4(__uint_as_float(v[0]) * p.scale, __uint_as_float(v[1]) * p.scale,
+                               __uint_as_float(v[2]) * p.scale, __uint_as_float(v[3]) * p.scale);
+          }
+          transpose8(e, lane);                     // lane 8G + k: chunk k of rows 8G .. 8G + 7
+          const int col = j0 + 32 * blk + 4 * k;
+          if (col < p.nb) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+              const int i = row0 + 8 * grp + r;
+              if (i < p.nb) *reinterpret_cast<float4*>(base + (long long)i * p.nb + col) = e[r];
             }
-          ptx::fence_proxy_async_smem();             // generic writes -> TMA reads
-          __syncwarp();
-          if (lane == 0) {
-            for (int q = 0; q < 2; ++q)
-              if (32 * q < nv) ptx::tma_store_3d(&p.tm_out, st + q * kOutBox, j0 + 32 * q, 128 * rt + 32 * quad, h);
-            ptx::bulk_commit();
           }
         }
-      } else if (nv > 0 && i < p.nb) {
-        float* dst = p.out + ((long long)h * p.nb + i) * p.nb + j0;
+      } else {
+        const int i = row0 + lane;
+        if (i < p.nb) {
+          float* dst = base + (long long)i * p.nb + j0;
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < nv) dst[c] = __uint_as_float(sr[c]) * p.scale;
+          for (int c = 0; c < 64; ++c)
+            if (c < nv) dst[c] = __uint_as_float(sr[c]) * p.scale;
+        }
       }
     }
-    if (OUT_TMA && lane == 0) ptx::bulk_wait0();     // stores complete before the CTA exits
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -395,16 +425,6 @@ cudaError_t launch_softmax_rows(float* s, long long rows, int nb, cudaStream_t s
   return cudaGetLastError();
 }
 
-bool map_scores(CUtensorMap* m, float* base, int heads, int nb) {
-  cuuint64_t dims[3] = {(cuuint64_t)nb, (cuuint64_t)nb, (cuuint64_t)heads};
-  cuuint64_t strides[2] = {(cuuint64_t)nb * 4, (cuuint64_t)nb * nb * 4};
-  cuuint32_t box[3] = {32, 32, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 cudaError_t launch_estimate_tc(const float* qm, const float* km, float* out, int heads, int nb, int d, int* status,
@@ -425,15 +445,13 @@ cudaError_t launch_estimate_tc(const float* qm, const float* km, float* out, int
   tp.status = status;
   tp.timeout_ns = device_wait_timeout_ns();
   static_assert(kSmem <= 232448, "shared memory budget");
-  // TMA stores need 16-byte row strides and a 16-byte aligned base
-  const bool out_tma = nb % 4 == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0 &&
-                       map_scores(&tp.tm_out, out, heads, nb);
-  cudaError_t e = cudaFuncSetAttribute(out_tma ? estimate_tc_kernel<true> : estimate_tc_kernel<false>,
+  const bool vec = nb % 4 == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
+  cudaError_t e = cudaFuncSetAttribute(vec ? estimate_tc_kernel<true> : estimate_tc_kernel<false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   const int grid = tp.n_items < num_sms() ? tp.n_items : num_sms();
   if (grid <= 0) return cudaSuccess;
-  if (out_tma) estimate_tc_kernel<true><<<grid, kThreads, kSmem, s>>>(tp);
+  if (vec) estimate_tc_kernel<true><<<grid, kThreads, kSmem, s>>>(tp);
   else estimate_tc_kernel<false><<<grid, kThreads, kSmem, s>>>(tp);
   e = cudaGetLastError();
   if (e != cudaSuccess || !probs) return e;

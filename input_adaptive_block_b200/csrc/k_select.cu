@@ -104,7 +104,7 @@ __device__ __forceinline__ int find_bin(const uint32_t* bins, uint32_t r, int la
 // SCORES: `in` holds scores (softmax formed here) instead of probabilities.
 // vec: rows of `in` and `idx` are 16-byte aligned (nb % 4 == 0).
 template <int NPL, bool WIN, bool SCORES>
-__global__ void __launch_bounds__(kSelWarps * 32, 6) select_kernel(const float* __restrict__ in,
+__global__ void __launch_bounds__(kSelWarps * 32, NPL > 24 ? 6 : 8) select_kernel(const float* __restrict__ in,
                                                                   const __grid_constant__ SelectTaus taus,
                                                                   int* __restrict__ cnt, int* __restrict__ idx,
                                                                   int heads, int nb, int vec) {
