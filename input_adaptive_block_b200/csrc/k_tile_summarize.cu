@@ -147,6 +147,98 @@ __global__ void __launch_bounds__(256, 5) summarize_kernel(const uint8_t* __rest
   }
 }
 
+// Wide form (bf16): lane owns the two adjacent 16-byte chunks 2l, 2l+1 of a
+// group of 64 (a warp covers 1 KB of the token row) and reads both with one
+// 32-byte load per token: half the load instructions and pointer steps per
+// byte.  Used when every row start is 32-byte aligned.
+__device__ __forceinline__ void ld32(uint4& a, uint4& b, const uint8_t* p) {
+  asm volatile("ld.global.nc.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+               : "l"(p));
+}
+
+template <bool BF16, int MODE>
+__global__ void __launch_bounds__(256, 4) summarize_wide_kernel(const uint8_t* __restrict__ in0,
+                                                              const uint8_t* __restrict__ in1,
+                                                              float* __restrict__ out0, float* __restrict__ out1,
+                                                              Geo g, long long row_bytes, int head_off_bytes,
+                                                              int chunks, int d) {
+  constexpr int EPC = BF16 ? 8 : 4;  // elements per 16-byte chunk
+  const int lane = threadIdx.x & 31;
+  const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int groups = (chunks + 63) / 64;
+  const long long n_units = (long long)g.nb * groups;
+  const long long all_units = in1 ? 2 * n_units : n_units;
+  const long long sy = (long long)g.W * row_bytes;     // next y row
+  const long long st = (long long)g.H * sy;            // next frame
+  for (long long uu = gwarp; uu < all_units; uu += nwarps) {
+    const bool second = uu >= n_units;
+    const long long u = second ? uu - n_units : uu;
+    const uint8_t* x = second ? in1 : in0;
+    float* out = second ? out1 : out0;
+    const int b = (int)(u / groups);
+    const int c = (int)(u - (long long)b * groups) * 64 + 2 * lane;   // first of the lane's two chunks
+    int t0, y0, x0, et, eh, ew;
+    block_box(g, b, t0, y0, x0, et, eh, ew);
+    const int nvalid = et * eh * ew;
+    float acc0[EPC], acc1[EPC];
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) acc0[e] = acc1[e] = MODE == 0 ? 0.f : (MODE == 1 ? -INFINITY : INFINITY);
+    if (c < chunks) {
+      const uint8_t* ptr = x + head_off_bytes + (long long)c * 16 +
+                           (((long long)t0 * g.H + y0) * g.W + x0) * row_bytes;
+      const long long wrap_y = sy - (long long)ew * row_bytes;
+      const long long wrap_t = st - (long long)eh * sy;
+      int xl = 0, yl = 0;
+      auto step = [&]() {
+        ptr += row_bytes;
+        if (++xl == ew) {
+          xl = 0;
+          ptr += wrap_y;
+          if (++yl == eh) {
+            yl = 0;
+            ptr += wrap_t;
+          }
+        }
+      };
+      int i = 0;
+      for (; i + 4 <= nvalid; i += 4) {
+        uint4 va[4], vb[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          ld32(va[r], vb[r], ptr);
+          step();
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          accumulate<BF16, MODE>(acc0, va[r]);
+          accumulate<BF16, MODE>(acc1, vb[r]);
+        }
+      }
+      for (; i < nvalid; ++i) {
+        uint4 va, vb;
+        ld32(va, vb, ptr);
+        accumulate<BF16, MODE>(acc0, va);
+        accumulate<BF16, MODE>(acc1, vb);
+        step();
+      }
+      const float inv = MODE == 0 ? 1.0f / (float)nvalid : 1.0f;
+      const int e0 = c * EPC;             // element index within the head-range row (both chunks in one head)
+      const int h = e0 / d, dd = e0 - h * d;
+      float4* o = reinterpret_cast<float4*>(out + ((long long)h * g.nb + b) * d + dd);
+      o[0] = make_float4(acc0[0] * inv, acc0[1] * inv, acc0[2] * inv, acc0[3] * inv);
+      if (BF16) {
+        o[1] = make_float4(acc0[4] * inv, acc0[5] * inv, acc0[6] * inv, acc0[7] * inv);
+        o[2] = make_float4(acc1[0] * inv, acc1[1] * inv, acc1[2] * inv, acc1[3] * inv);
+        o[3] = make_float4(acc1[4] * inv, acc1[5] * inv, acc1[6] * inv, acc1[7] * inv);
+      } else {
+        o[1] = make_float4(acc1[0] * inv, acc1[1] * inv, acc1[2] * inv, acc1[3] * inv);
+      }
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_tile3d(const void* x, void* xt, const Geo& g, int heads, int d, spade_dtype dt,
@@ -166,15 +258,23 @@ cudaError_t launch_summarize_m(const void* x0, const void* x1, float* out0, floa
   const int esz = dt == SPADE_BF16 ? 2 : 4;
   const long long row_bytes = (long long)heads_total * d * esz;
   const int chunks = hc * d * esz / 16;
-  const int groups = (chunks + 31) / 32;
+  const uint8_t* a = static_cast<const uint8_t*>(x0);
+  const uint8_t* b = static_cast<const uint8_t*>(x1);
+  const long long head_off = (long long)h0 * d * esz;
+  const bool wide = dt == SPADE_BF16 && row_bytes % 32 == 0 && head_off % 32 == 0 &&
+                    (reinterpret_cast<uintptr_t>(a) & 31) == 0 && (!b || (reinterpret_cast<uintptr_t>(b) & 31) == 0);
+  const int groups = wide ? (chunks + 63) / 64 : (chunks + 31) / 32;
   const long long units = (long long)g.nb * groups * (x1 ? 2 : 1);
-  const long long resident = 5LL * num_sms() * 8;      // warps
+  const long long resident = (wide ? 4LL : 5LL) * num_sms() * 8;      // warps
   const long long per_warp = (units + resident - 1) / resident;
   const long long warps = (units + per_warp - 1) / per_warp;
   long long blocks = (warps + 7) / 8;
   if (blocks < 1) blocks = 1;
-  const uint8_t* a = static_cast<const uint8_t*>(x0);
-  const uint8_t* b = static_cast<const uint8_t*>(x1);
+  if (wide) {
+    summarize_wide_kernel<true, MODE><<<(int)blocks, 256, 0, s>>>(a, b, out0, out1, g, row_bytes, (int)head_off,
+                                                                   chunks, d);
+    return cudaGetLastError();
+  }
   if (dt == SPADE_BF16)
     summarize_kernel<true, MODE><<<(int)blocks, 256, 0, s>>>(a, b, out0, out1, g, row_bytes, h0 * d * esz, chunks, d);
   else
