@@ -578,6 +578,7 @@ def main(argv=None):
     if rank == 0:
         line = assemble_line(value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
                              ms=ms, config=workload_config(wl, tau), extra=extra)
+        line["dtype"] = "f32" if wl.dtype == "f32" else "bf16"   # the arithmetic type the path runs in
         print(json.dumps(line))
     if world > 1:
         dist.barrier()

@@ -209,3 +209,61 @@ def test_exp2_polynomial_against_exp2():
     assert rel <= 1e-4, rel
     lo = api.selftest_exp2_poly(torch.tensor([-126.0, -200.0, -1e30, -float("inf")], device="cuda")).cpu()
     assert (lo >= 0).all() and (lo <= 2.0 ** -124).all(), lo
+
+
+def _geometric_row(rng, nb, n, total=1.0, skip=()):
+    """n well-separated values total * 2^-(k+1) (k = 0..n-1, renormalised to
+    `total`) at random positions outside `skip`; zeros elsewhere."""
+    row = np.zeros(nb, np.float64)
+    cols = [j for j in rng.permutation(nb) if j not in set(skip)][:n]
+    vals = 0.5 ** (np.arange(n) + 1)
+    row[cols] = vals / vals.sum() * total
+    return row
+
+
+@pytest.mark.parametrize("nb", [40, 660])
+def test_select_degenerate_rows(nb):
+    """Rows the index search must handle besides softmax output: exact zeros,
+    a diagonal that alone reaches tau, a row summing to more than 1 (masses
+    scaled per row), NaN / negative / above-1 entries (clamped to [0, 1], NaN
+    counted as 0), an all-zero row (the mass never reaches tau: every block
+    kept), and with a tiny tau a zero diagonal (one more block needed) and a
+    non-zero one (the diagonal alone).  Values are powers of two far from the
+    cut, so the oracle on the clamped row gives the one correct answer."""
+    rng = np.random.default_rng(nb)
+    P = np.stack([np.stack([_geometric_row(rng, nb, 30) for _ in range(nb)]) for _ in range(2)])
+    special = {}
+    # head 0, tau = 0.9
+    special[(0, 0)] = _geometric_row(rng, nb, 20, skip=(0,))                  # zero diagonal, zeros elsewhere
+    r = _geometric_row(rng, nb, 12, total=0.05, skip=(1,)); r[1] = 0.95
+    special[(0, 1)] = r                                                        # the diagonal alone reaches tau
+    special[(0, 2)] = _geometric_row(rng, nb, 16, total=1.7)                   # sums to 1.7
+    r = _geometric_row(rng, nb, 16)
+    others = [j for j in range(nb) if r[j] == 0 and j != 3]
+    r[others[:3]] = np.nan
+    r[others[3:6]] = -0.5
+    special[(0, 3)] = r                                                        # NaN and negative entries
+    r = _geometric_row(rng, nb, 16, total=0.3, skip=(4,))
+    r[[j for j in range(nb) if r[j] == 0 and j != 4][0]] = 3.0
+    special[(0, 4)] = r                                                        # an entry above 1
+    special[(0, 5)] = np.zeros(nb)                                             # all zero
+    # head 1, tau = 1e-6
+    special[(1, 0)] = _geometric_row(rng, nb, 20, skip=(0,))                  # zero diagonal
+    r = _geometric_row(rng, nb, 20, skip=(1,)); r[1] = 1e-3
+    special[(1, 1)] = r                                                        # small non-zero diagonal
+    for (h, i), row in special.items():
+        P[h, i] = row
+    taus = [0.9, 1e-6]
+    cnt, idx = api.select(torch.tensor(P, dtype=torch.float32).cuda(), taus)
+    cnt, idx = cnt.cpu().numpy(), idx.cpu().numpy()
+    for (h, i), row in special.items():
+        clamped = np.clip(np.nan_to_num(row.astype(np.float32).astype(np.float64), nan=0.0), 0.0, 1.0)
+        want = O.select_row(clamped, i, taus[h])
+        got = list(map(int, idx[h, i, : cnt[h, i]]))
+        assert got == want, (h, i, got, want)
+    assert cnt[0, 5] == nb and cnt[0, 1] == 1 and cnt[1, 1] == 1 and cnt[1, 0] == 2
+    # every other row: ascending, diagonal present, ids in range
+    for h in range(2):
+        for i in range(nb):
+            g = list(idx[h, i, : cnt[h, i]])
+            assert g == sorted(set(g)) and i in g and all(0 <= j < nb for j in g)
