@@ -108,6 +108,22 @@ def test_estimate_scores_random_many_blocks():
         assert np.abs(S - ref).max() <= SCORE_REL * max(1.0, np.abs(ref).max()), d
 
 
+@pytest.mark.parametrize("nb", [2047, 2048])
+def test_estimate_at_the_block_limit(nb):
+    """nb at the estimator's limit (2048: 16 key tiles per row, the widest
+    row-softmax variant) and one below it (ragged last tile, rows not
+    16-byte aligned)."""
+    g = torch.Generator(device="cpu").manual_seed(nb)
+    qm = (torch.randn(2, nb, 64, generator=g) * 0.6).cuda()
+    km = (torch.randn(2, nb, 64, generator=g) * 0.6).cuda()
+    S = to_np(api.estimate_scores(qm, km))
+    ref = O.pooled_scores(to_np(qm), to_np(km))
+    assert np.abs(S - ref).max() <= SCORE_REL * max(1.0, np.abs(ref).max())
+    P = to_np(api.estimate(qm, km))
+    assert np.abs(P - O.softmax_rows(ref)).max() <= PROB_ABS
+    assert np.abs(P.sum(-1) - 1).max() <= 1e-5
+
+
 @pytest.mark.parametrize("wl", RAGGED + [get_config("wan1.3b")], ids=lambda w: w.name)
 def test_select_scores_against_oracle_chain(wl):
     """The grouped path's steps 3-4 (scores, then the softmax fused into the
