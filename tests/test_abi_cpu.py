@@ -148,3 +148,33 @@ def test_copy_head_slice_host_validation():
     assert lib.spade_copy_head_slice(None, fake, 10, 4, 0, 2, 128, 1, 1, None) == _lib.SPADE_ERR_INVALID
     assert lib.spade_copy_head_slice(fake, fake, 10, 4, 3, 2, 128, 1, 1, None) == _lib.SPADE_ERR_INVALID
     assert lib.spade_copy_head_slice(fake, fake, 0, 4, 0, 2, 128, 1, 1, None) == _lib.SPADE_ERR_INVALID
+
+
+def test_fused_form_entry_points_host_validation():
+    """spade_summarize_qk, spade_estimate_scores and spade_select_scores reject
+    bad arguments on the host, before anything is enqueued."""
+    lib = _lib.load()
+    fake = ctypes.c_void_p(1 << 20)                 # never dereferenced: validation fails first
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    g = SpadeGeom(21, 45, 80, 2, 8, 8)
+    # summarize_qk: null / misaligned pointers, bad d, bad geometry, no heads
+    assert lib.spade_summarize_qk(None, fake, fake, fake, g, 4, 128, 1, None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_summarize_qk(fake, fake, odd, fake, g, 4, 128, 1, None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_summarize_qk(fake, fake, fake, fake, g, 4, 96, 1, None) == _lib.SPADE_ERR_UNSUPPORTED
+    assert lib.spade_summarize_qk(fake, fake, fake, fake, SpadeGeom(0, 1, 1, 1, 1, 1), 4, 128, 1,
+                                  None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_summarize_qk(fake, fake, fake, fake, g, 0, 128, 1, None) == _lib.SPADE_ERR_INVALID
+    # estimate_scores: the same limits as spade_estimate
+    assert lib.spade_estimate_scores(None, fake, fake, 1, 10, 128, None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_estimate_scores(fake, fake, odd, 1, 10, 128, None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_estimate_scores(fake, fake, fake, 1, 4096, 128, None) == _lib.SPADE_ERR_UNSUPPORTED
+    assert lib.spade_estimate_scores(fake, fake, fake, 1, 10, 96, None) == _lib.SPADE_ERR_UNSUPPORTED
+    assert lib.spade_estimate_scores(fake, fake, fake, 0, 10, 128, None) == _lib.SPADE_ERR_INVALID
+    # select_scores: the same limits as spade_select
+    taus = (ctypes.c_float * 2)(0.9, 0.9)
+    bad_tau = (ctypes.c_float * 2)(0.9, float("nan"))
+    assert lib.spade_select_scores(None, taus, fake, fake, 2, 10, None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_select_scores(fake, taus, fake, fake, 2, 2000, None) == _lib.SPADE_ERR_UNSUPPORTED
+    assert lib.spade_select_scores(fake, taus, fake, fake, 2, 0, None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_select_scores(fake, bad_tau, fake, fake, 2, 10, None) == _lib.SPADE_ERR_INVALID
+    assert lib.spade_select_scores(fake, taus, fake, fake, 2000, 10, None) == _lib.SPADE_ERR_UNSUPPORTED
