@@ -15,11 +15,12 @@
 //
 //  * Persistent CTAs, each over a contiguous range of items (head, 128 query
 //    rows, 128 key columns), so the query tile changes only a few times per
-//    CTA.  The query tile lives in TMEM: a converter warpgroup (thread =
-//    query row) reads it from global memory (the next 32 columns' loads in
-//    flight while the current ones are split), splits it and writes Qhi and
-//    Qlo with tcgen05.st; the MMAs read them as the A operand, so only key
-//    chunks pass through shared memory.  Per item and 32-element d chunk:
+//    CTA.  The query tile lives in TMEM: its fp32 chunks come through the
+//    stage ring ahead of time (TMA), and once the previous tile's MMAs are
+//    done a converter warpgroup (thread = query row) splits them and writes
+//    Qhi and Qlo with tcgen05.st; the MMAs read them as the A operand, so
+//    only key chunks pass through shared memory as operands.  Per item and
+//    32-element d chunk:
 //    TMA loads the fp32 K chunk (128 rows x 128 B, 128-byte swizzled: the
 //    K-major layout the MMA reads) into one of six stages; the converter
 //    rewrites it as hi in place and lo beside it (elementwise, so the
@@ -51,8 +52,8 @@ constexpr int kSmem = kStages * kStageBytes + 256 + 1024;
 constexpr uint32_t kColQhi = 256, kColQlo = 384;
 
 struct __align__(64) EstTcParams {
-  CUtensorMap tm_k;         // [heads][nb][d] fp32: dims {d, nb, heads}, box {32, 128, 1}
-  const float* qm;          // [heads][nb][d] fp32
+  CUtensorMap tm_q;         // [heads][nb][d] fp32: dims {d, nb, heads}, box {32, 128, 1}
+  CUtensorMap tm_k;         // same for the key means
   float* out;               // [heads][nb][nb] scores
   int nb, d, nt, n_items;
   float scale;
@@ -99,43 +100,6 @@ __device__ __forceinline__ uint32_t idesc_tf32(uint32_t n) {
 __device__ __forceinline__ uint32_t tf32_hi(uint32_t x) { return x & 0xFFFFE000u; }
 __device__ __forceinline__ uint32_t tf32_lo(uint32_t x) {
   return __float_as_uint(__uint_as_float(x) - __uint_as_float(tf32_hi(x)));
-}
-__device__ __forceinline__ uint32_t tf32_hi(float x) { return tf32_hi(__float_as_uint(x)); }
-__device__ __forceinline__ uint32_t tf32_lo(float x) { return tf32_lo(__float_as_uint(x)); }
-
-__device__ __forceinline__ void load8(float4 (&v)[8], const float4* src, bool valid) {
-#pragma unroll
-  for (int q = 0; q < 8; ++q) v[q] = valid ? __ldg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-}
-
-// Rows 32*(warp&3) .. +31 of the query tile (head h, tile rt) into TMEM as
-// TF32 hi / lo: one row per thread, 32 columns per tcgen05.st, the next 32
-// columns' loads in flight while the current ones are split and stored.
-__device__ __forceinline__ void load_q_tile(const EstTcParams& p, int h, int rt, int quad, int lane, uint32_t tmem) {
-  const int i = 128 * rt + quad * 32 + lane;
-  const bool valid = i < p.nb;
-  const float4* src = reinterpret_cast<const float4*>(p.qm + ((long long)h * p.nb + (valid ? i : 0)) * p.d);
-  const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-  float4 cur[8], nxt[8];
-  load8(cur, src, valid);
-  for (int c0 = 0; c0 < p.d; c0 += 32) {
-    if (c0 + 32 < p.d) load8(nxt, src + (c0 + 32) / 4, valid);
-    uint32_t r[32];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      r[4 * q] = tf32_hi(cur[q].x); r[4 * q + 1] = tf32_hi(cur[q].y);
-      r[4 * q + 2] = tf32_hi(cur[q].z); r[4 * q + 3] = tf32_hi(cur[q].w);
-    }
-    ptx::tmem_st32(tmem + lane_base + kColQhi + c0, r);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      r[4 * q] = tf32_lo(cur[q].x); r[4 * q + 1] = tf32_lo(cur[q].y);
-      r[4 * q + 2] = tf32_lo(cur[q].z); r[4 * q + 3] = tf32_lo(cur[q].w);
-    }
-    ptx::tmem_st32(tmem + lane_base + kColQlo + c0, r);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) cur[q] = nxt[q];
-  }
 }
 
 __device__ __forceinline__ float4 shfl_xor4(float4 v, int m) {
@@ -195,7 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) ptx::prefetch_tmap(&p.tm_k);
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&p.tm_q);
+    ptx::prefetch_tmap(&p.tm_k);
+  }
   if (warp == 1) {
     ptx::tmem_alloc(tmem_slot, 512);
     ptx::tmem_relinquish();
@@ -216,13 +183,17 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     uint32_t g = 0;
     bool ok = true;
     for (int it = it0; ok && it < it1; ++it) {
-      const int h = it / (nt * nt), ct = it % nt;
-      for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
+      const int h = it / (nt * nt), rt = (it / nt) % nt, ct = it % nt;
+      // a new query tile: its d chunks go through the ring first (read into
+      // TMEM by the converter), then the item's key chunks
+      const bool qt = it == it0 || ct == 0;
+      for (int k = qt ? 0 : ndc; ok && k < 2 * ndc; ++k, ++g) {
         const int s = (int)(g % kStages);
         ok = __all_sync(0xffffffffu, ewait(&empty[s], ((g / kStages) & 1) ^ 1, W));
         if (!ok) break;
         ptx::mbar_arrive_expect_tx_elect(&full[s], kChunk);
-        ptx::tma_load_3d_elect(smem + s * kStageBytes, &p.tm_k, &full[s], 32 * dc, 128 * ct, h);
+        if (k < ndc) ptx::tma_load_3d_elect(smem + s * kStageBytes, &p.tm_q, &full[s], 32 * k, 128 * rt, h);
+        else ptx::tma_load_3d_elect(smem + s * kStageBytes, &p.tm_k, &full[s], 32 * (k - ndc), 128 * ct, h);
       }
     }
     if (lane == 0 && !ok && g > 0) {   // wind down: let the loads issued land
@@ -236,6 +207,14 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     for (int it = it0; ok && it < it1; ++it, ++gi) {
       if (it == it0 || it % nt == 0) {                 // a new query tile
         if (gq > 0) ptx::tc_commit_elect(q_free);      // fires once the previous tile's MMAs are done
+        // its chunks' stages: read into TMEM by the converter, then released here
+        for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
+          const int s = (int)(g % kStages);
+          ok = __all_sync(0xffffffffu, ewait(&conv[s], (g / kStages) & 1, W));
+          if (!ok) break;
+          if (lane == 0) ptx::mbar_arrive(&empty[s]);
+        }
+        if (!ok) break;
         ok = __all_sync(0xffffffffu, ewait(q_full, gq & 1, W));
         if (!ok) break;
         ptx::tc_fence_after();
@@ -278,12 +257,40 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
     bool ok = true;
     for (int it = it0; ok && it < it1; ++it) {
       if (it == it0 || it % nt == 0) {
+        // the new query tile's chunks have been loaded into the ring ahead of
+        // time; once the previous tile's MMAs are done, thread = query row
+        // reads its row of each chunk (128-byte swizzled: 16-byte chunk c at
+        // position c ^ (row & 7)), splits it and writes Qhi / Qlo to TMEM
         if (gq > 0) {
           ok = ewait(q_free, (gq - 1) & 1, W);         // the previous tile's MMAs have read it
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           ptx::tc_fence_after();
         }
-        load_q_tile(p, it / (nt * nt), (it / nt) % nt, quad, lane, tmem);
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        for (int dc = 0; ok && dc < ndc; ++dc, ++g) {
+          const int s = (int)(g % kStages);
+          ok = ewait(&full[s], (g / kStages) & 1, W);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          const uint8_t* rowp = smem + s * kStageBytes + ctid * 128;
+          uint4 v[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(rowp + ((c ^ (ctid & 7)) << 4));
+          uint32_t r[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            r[4 * c] = tf32_hi(v[c].x); r[4 * c + 1] = tf32_hi(v[c].y);
+            r[4 * c + 2] = tf32_hi(v[c].z); r[4 * c + 3] = tf32_hi(v[c].w);
+          }
+          ptx::tmem_st32(tmem + lane_base + kColQhi + 32 * dc, r);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            r[4 * c] = tf32_lo(v[c].x); r[4 * c + 1] = tf32_lo(v[c].y);
+            r[4 * c + 2] = tf32_lo(v[c].z); r[4 * c + 3] = tf32_lo(v[c].w);
+          }
+          ptx::tmem_st32(tmem + lane_base + kColQlo + 32 * dc, r);
+          ptx::mbar_arrive(&conv[s]);                  // stage read: the MMA warp releases it
+        }
+        if (!ok) break;
         ptx::tc_fence_before();
         ptx::mbar_arrive(q_full);
         ++gq;
@@ -434,8 +441,7 @@ cudaError_t launch_estimate_tc(const float* qm, const float* km, float* out, int
     return cudaErrorInvalidValue;
   static EstTcParams tp;
   memset(&tp, 0, sizeof(tp));
-  if (!map_means(&tp.tm_k, km, heads, nb, d)) return cudaErrorInvalidValue;
-  tp.qm = qm;
+  if (!map_means(&tp.tm_q, qm, heads, nb, d) || !map_means(&tp.tm_k, km, heads, nb, d)) return cudaErrorInvalidValue;
   tp.out = out;
   tp.nb = nb;
   tp.d = d;
