@@ -44,11 +44,7 @@ constexpr uint32_t kOneKey = 0x3F800000u;  // bit pattern of 1.0f, the largest k
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr float kMassOne = 1073741824.0f;  // 2^30: fixed-point mass of probability 1
 
-__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
-  return v;
-}
+__device__ __forceinline__ uint32_t warp_sum(uint32_t v) { return __reduce_add_sync(kFull, v); }
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
@@ -117,17 +113,20 @@ __global__ void __launch_bounds__(kSelWarps * 32, NPL > 24 ? 6 : 8) select_kerne
   const int i = (int)(row - (long long)h * nb);
   const float* prow = in + row * nb;
   const int j0 = lane * NPL;
+  // blocks past nb read as -inf (scores: exp gives 0) or 0 (probabilities),
+  // so the passes below need no per-block range test
+  const float pad = SCORES ? -INFINITY : 0.f;
   float x[NPL];
   if (vec) {
 #pragma unroll
     for (int q = 0; q < NPL / 4; ++q) {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 v = make_float4(pad, pad, pad, pad);
       if (j0 + 4 * q < nb) v = __ldg(reinterpret_cast<const float4*>(prow + j0) + q);
       x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
     }
   } else {
 #pragma unroll
-    for (int e = 0; e < NPL; ++e) x[e] = j0 + e < nb ? __ldg(prow + j0 + e) : 0.f;
+    for (int e = 0; e < NPL; ++e) x[e] = j0 + e < nb ? __ldg(prow + j0 + e) : pad;
   }
   uint32_t* bins = sbin[warp];
   zero_bins(bins, lane);                           // while the row is in flight
@@ -136,13 +135,12 @@ __global__ void __launch_bounds__(kSelWarps * 32, NPL > 24 ? 6 : 8) select_kerne
     // the Estimator's softmax over the row's valid key blocks: p_j = x_j * pmul
     float mx = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < NPL; ++e)
-      if (j0 + e < nb) mx = fmaxf(mx, x[e]);
+    for (int e = 0; e < NPL; ++e) mx = fmaxf(mx, x[e]);
     mx = warp_max(mx);
     float l = 0.f;
 #pragma unroll
     for (int e = 0; e < NPL; ++e) {
-      const float t = j0 + e < nb ? __expf(x[e] - mx) : 0.f;
+      const float t = __expf(x[e] - mx);          // 0 past nb
       x[e] = t;
       l += t;
     }
@@ -181,10 +179,10 @@ __global__ void __launch_bounds__(kSelWarps * 32, NPL > 24 ? 6 : 8) select_kerne
         if (++jy == taus.nbh) { jy = 0; ++jt; }
       }
     }
-    const float p = SCORES ? fminf(x[e] * pmul, 1.0f) : x[e];   // 0 past nb
+    const float p = SCORES ? x[e] * pmul : x[e];   // <= 1 (a product of two values <= 1); 0 past nb
     const uint32_t m = __float2uint_rn(p * scale);
     uint32_t k = 0u;
-    if (j < nb && in_win) {
+    if ((WIN ? j < nb : true) && in_win) {         // without a window, j == i < nb
       win |= 1u << e;
       dl += m;
     } else if (m > 0u) {                           // massless blocks are never needed
