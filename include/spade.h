@@ -39,6 +39,11 @@
  *    are latched in a device status word, readable with
  *    spade_last_device_status().
  *  - Pointers must be 16-byte aligned.  bf16 = IEEE bfloat16 bit pattern.
+ *  - Several host threads may call the library at once: each call stages its
+ *    launch parameters in storage of its own thread, and the launch copies
+ *    them.  The GPU-side rules are the caller's: calls whose buffers (or,
+ *    for spade_block_sparse_attn_noalloc, the library's fixed scratch)
+ *    overlap must be ordered on the GPU (one stream, or events).
  */
 #ifndef SPADE_H_
 #define SPADE_H_
@@ -204,8 +209,9 @@ spade_status spade_block_sparse_attn(const void* q, const void* k, const void* v
  *    capture.
  *  - Every call shares the one array, and each call rewrites it in full
  *    (the counter is reset on the device at the start of each call).  Calls
- *    whose work overlaps on the GPU -- on different streams, or from
- *    different threads -- race on it; order them (one stream, or events). */
+ *    from any host threads may be made, but calls whose work overlaps on the
+ *    GPU (on different streams) race on the array; order them (one stream,
+ *    or events). */
 spade_status spade_block_sparse_attn_noalloc(const void* q, const void* k, const void* v, void* out,
                                              const int* cnt, const int* idx, spade_geom g,
                                              int heads, int d, int text_tokens, spade_dtype dt,
@@ -295,17 +301,6 @@ spade_status spade_last_device_status(spade_stream_t stream);
 const char* spade_status_string(spade_status s);
 const char* spade_last_error_message(void);   /* detail of the last host error */
 int spade_version(void);
-
-/* Runs a kernel whose single wait can never be satisfied, bounded by
- * timeout_ns; the device status must then read SPADE_ERR_TIMEOUT.  Exercises
- * the bounded-wait error path without faulting or hanging the GPU. */
-spade_status spade_selftest_bounded_wait(int64_t timeout_ns, spade_stream_t stream);
-
-/* Evaluates, for n device floats x (x <= 8), the polynomial 2^x the attention
- * kernel uses for part of its softmax exponentials (round-to-nearest range
- * reduction, cubic on [-1/2, 1/2]; relative error <= 1e-4 for x >= -125,
- * inputs below -125 are clamped).  y: n device floats.  For testing. */
-spade_status spade_selftest_exp2_poly(const float* x, float* y, int n, spade_stream_t stream);
 
 #ifdef __cplusplus
 }

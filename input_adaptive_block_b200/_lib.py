@@ -63,7 +63,6 @@ SIGNATURES = {
     "spade_last_error_message": (ctypes.c_char_p, []),
     "spade_version": (c_int, []),
     "spade_selftest_bounded_wait": (c_int, [c_int64, c_void_p]),
-    "spade_selftest_exp2_poly": (c_int, [c_void_p, c_void_p, c_int, c_void_p]),
 }
 
 _lib = None

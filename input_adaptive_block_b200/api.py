@@ -357,13 +357,6 @@ def last_device_status(stream=None) -> int:
     return int(_lib.load().spade_last_device_status(_stream(stream)))
 
 
-def selftest_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
-    y = torch.empty_like(x)
-    check(_lib.load().spade_selftest_exp2_poly(_dev(x, "x"), _dev(y, "y"), x.numel(), _stream(stream)),
-          "spade_selftest_exp2_poly")
-    return y
-
-
 def selftest_bounded_wait(timeout_ns: int, stream=None) -> None:
     check(_lib.load().spade_selftest_bounded_wait(int(timeout_ns), _stream(stream)),
           "spade_selftest_bounded_wait")

@@ -58,8 +58,7 @@ constexpr int kItemRing = 4;                 // work items in flight between the
 constexpr uint32_t kFullBlock = 1u << 31;    // extent code: every slot valid (low bits = 128)
 constexpr int kEdgeCases = 8;                // key/value maps per scheme: bit 0 t-, bit 1 y-, bit 2 x-edge
 
-// POLY_: when 1, every fourth column pair's exponential runs on the FMA pipe
-template <int D, int NS_, int POLY_>
+template <int D, int NS_>
 struct Cfg {
   static constexpr int TILE = 128 * D * 2;
   // K/V ring stages (TMA latency under load is ~1-1.5 us, so the ring holds
@@ -276,37 +275,15 @@ __device__ __forceinline__ uint32_t extent_code(const TcParams& p, const Item& I
   return (uint32_t)valid | (valid >= 128 ? kFullBlock : 0u);
 }
 
-// ------------------------------------------------------- exp2 on the FMA pipe --
-// 2^x for a pair of floats without the SFU.  Range reduction x = n + f with
-// n = round(x) obtained by adding 1.5 * 2^23 (the integer lands in the low
-// mantissa bits; Cody & Waite style reduction), |f| <= 1/2; 2^f by a cubic
-// fitted to 2^f on Chebyshev nodes of [-1/2, 1/2] (relative error <= 7.5e-5,
-// far below the bf16 rounding the result goes through); 2^n is added to the
-// exponent field with one integer multiply-add.  Inputs are clamped at -125
-// so that every result stays a normal float.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 j = __fadd2_rn(x, make_float2(kRound, kRound));
-  const float2 n = __fadd2_rn(j, make_float2(-kRound, -kRound));
-  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
-  float2 q = __ffma2_rn(make_float2(0.055171654f, 0.055171654f), f, make_float2(0.24261113f, 0.24261113f));
-  q = __ffma2_rn(q, f, make_float2(0.69326097f, 0.69326097f));
-  q = __ffma2_rn(q, f, make_float2(0.99992806f, 0.99992806f));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(j.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(j.y) << 23)));
-}
-
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
 
-template <int D, int NS, int POLY>
-__global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
-  using C = Cfg<D, NS, POLY>;
+template <int D, int NS>
+__global__ void __launch_bounds__(Cfg<D, NS>::THREADS, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
+  using C = Cfg<D, NS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
@@ -623,7 +600,7 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
         if (l != 0.f && m_seen != m_use) l *= ptx::ex2(m_seen - m_use);
         m_seen = m_use;
         // p = 2^(s*scale*log2e - m) in four 32-column chunks: FFMA2, exp2
-        // (SFU; with POLY, every fourth pair on the FMA pipe), row-sum FADD2,
+        // (SFU), row-sum FADD2,
         // bf16 pack, TMEM store; masked columns are -inf and give 0 (chunks
         // past a short block's prefix are computed all the same: a branch
         // between chunks costs more than it saves)
@@ -640,12 +617,8 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
                   make_float2(__uint_as_float(sr[32 * q + 2 * c]), __uint_as_float(sr[32 * q + 2 * c + 1])), sl2x2, nm2);
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-              if (POLY && (c & 3) == 3) {
-                pe[c] = exp2_poly2(pe[c]);
-              } else {
-                pe[c].x = ptx::ex2(pe[c].x);
-                pe[c].y = ptx::ex2(pe[c].y);
-              }
+              pe[c].x = ptx::ex2(pe[c].x);
+              pe[c].y = ptx::ex2(pe[c].y);
             }
 #pragma unroll
             for (int c = 0; c < 16; ++c) acc4[c & 3] = __fadd2_rn(acc4[c & 3], pe[c]);
@@ -744,15 +717,17 @@ __global__ void __launch_bounds__(Cfg<D, NS, POLY>::THREADS, 1) attn_tc_kernel(c
 }
 
 // ------------------------------------------------------------------ host --
+// The driver's tensor-map encoder, looked up once (initialisation of a
+// function-local static is thread-safe); null without a driver.
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+  }();
   return fn;
 }
 
@@ -781,21 +756,21 @@ bool map_text(CUtensorMap* m, const void* base, int text, int heads, int d) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int NS, int POLY>
+template <int D, int NS>
 cudaError_t launch_d(const TcParams& tp, int grid, cudaStream_t s) {
-  using C = Cfg<D, NS, POLY>;
+  using C = Cfg<D, NS>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
   static_assert(C::REG_POOL_NEEDED <= 65536, "register split");
   cudaError_t e =
-      cudaFuncSetAttribute(attn_tc_kernel<D, NS, POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+      cudaFuncSetAttribute(attn_tc_kernel<D, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   // The warpgroups' register increase waits for room in the block's
   // launch-time pool: never launch a build whose pool is smaller than the split.
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D, NS, POLY>);
+  e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D, NS>);
   if (e != cudaSuccess) return e;
   if (fa.numRegs * C::THREADS < C::REG_POOL_NEEDED) return cudaErrorNotSupported;
-  attn_tc_kernel<D, NS, POLY><<<grid, C::THREADS, C::SMEM, s>>>(tp);
+  attn_tc_kernel<D, NS><<<grid, C::THREADS, C::SMEM, s>>>(tp);
   return cudaGetLastError();
 }
 
@@ -814,7 +789,9 @@ bool attn_tc_supported(const AttnArgs& a) {
 }
 
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s, const char** why) {
-  static TcParams tp;   // host staging (large); launches copy it into the parameter buffer
+  // host staging (large), one per calling thread: the launch copies it into
+  // the kernel's parameter buffer, so concurrent callers never share it
+  thread_local TcParams tp;
   if (!encode_fn()) { *why = "cuTensorMapEncodeTiled unavailable"; return cudaErrorNotSupported; }
   memset(&tp, 0, sizeof(tp));
   const int es = 2;
@@ -863,8 +840,8 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s, const char** why) 
   tp.timeout_ns = device_wait_timeout_ns();
   const int grid = a.n_items < num_sms() ? a.n_items : num_sms();
   if (grid <= 0) return cudaSuccess;
-  if (a.d == 64) return launch_d<64, 8, 0>(tp, grid, s);
-  return launch_d<128, 5, 0>(tp, grid, s);
+  if (a.d == 64) return launch_d<64, 8>(tp, grid, s);
+  return launch_d<128, 5>(tp, grid, s);
 }
 
 // ------------------------------------------------- bounded-wait self test --
@@ -885,24 +862,6 @@ __global__ void bounded_wait_selftest_kernel(int* status, long long timeout_ns) 
 
 cudaError_t launch_bounded_wait_selftest(int* status, long long timeout_ns, cudaStream_t s) {
   bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(status, timeout_ns);
-  return cudaGetLastError();
-}
-
-// ------------------------------------------------ FMA-pipe exp2 self test --
-__global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
-    y[i] = r.x;
-    y[i + 1] = r.y;
-  } else if (i < n) {
-    y[i] = exp2_poly2(make_float2(x[i], 0.f)).x;
-  }
-}
-
-cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int n, cudaStream_t s) {
-  const int pairs = (n + 1) / 2;
-  exp2_poly_selftest_kernel<<<(pairs + 255) / 256, 256, 0, s>>>(x, y, n);
   return cudaGetLastError();
 }
 

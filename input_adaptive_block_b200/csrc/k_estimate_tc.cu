@@ -371,15 +371,17 @@ __global__ void __launch_bounds__(kThreads, 1) estimate_tc_kernel(const __grid_c
   if (warp == 1) ptx::tmem_dealloc(tmem, 512);
 }
 
+// The driver's tensor-map encoder, looked up once (initialisation of a
+// function-local static is thread-safe); null without a driver.
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+  }();
   return fn;
 }
 
@@ -439,7 +441,7 @@ cudaError_t launch_estimate_tc(const float* qm, const float* km, float* out, int
   if (!encode_fn()) return cudaErrorNotSupported;
   if (d % 32 != 0 || d > 128 || (reinterpret_cast<uintptr_t>(qm) & 15) || (reinterpret_cast<uintptr_t>(km) & 15))
     return cudaErrorInvalidValue;
-  static EstTcParams tp;
+  thread_local EstTcParams tp;   // per calling thread; the launch copies it
   memset(&tp, 0, sizeof(tp));
   if (!map_means(&tp.tm_q, qm, heads, nb, d) || !map_means(&tp.tm_k, km, heads, nb, d)) return cudaErrorInvalidValue;
   tp.out = out;

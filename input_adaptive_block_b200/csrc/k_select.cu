@@ -415,7 +415,9 @@ cudaError_t launch_select_t(const float* in, const SelectTaus& t, bool win, bool
 
 cudaError_t launch_select(const float* in, const float* tau_host, int* cnt, int* idx, int heads, int nb,
                           cudaStream_t s, const int* radius_host, const Geo* g, bool scores) {
-  static SelectTaus t;   // host staging (large); launches copy it into the parameter buffer
+  // host staging (large), one per calling thread: the launch copies it into
+  // the kernel's parameter buffer, so concurrent callers never share it
+  thread_local SelectTaus t;
   for (int h = 0; h < heads; ++h) t.tau[h] = tau_host[h];
   bool win = false;
   if (radius_host && g) {

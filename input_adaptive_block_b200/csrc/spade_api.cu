@@ -1,6 +1,7 @@
 // C ABI of the SPADE executor hot path (declared in include/spade.h):
 // argument validation, workspace layout, and the order of launches for the
 // single steps and for the grouped (mixed-scheme) layer.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -9,6 +10,7 @@
 #include <vector>
 
 #include "spade_internal.cuh"
+#include "spade_selftest.h"
 
 // Latched device status (SPADE_OK / SPADE_ERR_TIMEOUT), one per device.
 __device__ int g_spade_status;
@@ -47,16 +49,20 @@ int current_device() {
   return dev;
 }
 
+// Per-device caches below are atomics: callers on several host threads may
+// fill the same slot at once (with the same value).
 int* status_ptr() {
-  static int* ptrs[kMaxDevices] = {nullptr};
+  static std::atomic<int*> ptrs[kMaxDevices];
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_spade_status) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<int*>(p);
+  int* p = ptrs[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_spade_status) != cudaSuccess) return nullptr;
+    p = static_cast<int*>(a);
+    ptrs[dev].store(p, std::memory_order_release);
   }
-  return ptrs[dev];
+  return p;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -163,18 +169,36 @@ cudaError_t run_estimate(const float* qm, const float* km, float* out, int heads
   return e;
 }
 
+// Host checks of an attention launch that do not depend on pointers; every
+// entry point runs them before it enqueues anything.  A work item is packed
+// as (head << 16) | query block, so a head's query blocks (video blocks plus
+// text blocks) must number at most 65536; the CUDA-core kernel (taken when
+// the tensor-core kernel does not support the shape) holds at most 128 slots
+// per block.
+spade_status check_attention(const AttnArgs& a) {
+  const int ntb = text_blocks(a.text_tokens);
+  for (int h = 0; h < a.heads; ++h)
+    if ((long long)a.head[h].nb + ntb > 65536)
+      return fail(SPADE_ERR_UNSUPPORTED, "head %d: %d blocks + %d text blocks exceed 65536 query blocks", h,
+                  a.head[h].nb, ntb);
+  if (!attn_tc_supported(a))
+    for (int sc = 0; sc < a.n_schemes; ++sc)
+      if (a.geo[sc].bs > 128) return fail(SPADE_ERR_UNSUPPORTED, "CUDA-core attention needs blocks <= 128 slots");
+  return SPADE_OK;
+}
+
+// Enqueues the work list and the attention launch (check_attention has passed).
 spade_status run_attention(AttnArgs& a, cudaStream_t s) {
   a.status = status_ptr();
   if (!a.status) return fail(SPADE_ERR_CUDA, "device status word unavailable");
+  const bool tc = attn_tc_supported(a);
   cudaError_t e = launch_worklist(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "work list");
-  if (attn_tc_supported(a)) {
+  if (tc) {
     const char* why = "";
     e = launch_attn_tc(a, s, &why);
     if (e != cudaSuccess) return fail(SPADE_ERR_CUDA, "tensor-core attention: %s (%s)", cudaGetErrorString(e), why);
   } else {
-    for (int sc = 0; sc < a.n_schemes; ++sc)
-      if (a.geo[sc].bs > 128) return fail(SPADE_ERR_UNSUPPORTED, "CUDA-core attention needs blocks <= 128 slots");
     e = launch_attn_simt(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "CUDA-core attention");
   }
@@ -185,46 +209,48 @@ spade_status run_attention(AttnArgs& a, cudaStream_t s) {
 // a host-side stand-in in host code, so the address is looked up once per
 // device (with that device current) and cached.
 int* noalloc_scratch(spade_status* st) {
-  static int* ptrs[kMaxDevices] = {nullptr};
+  static std::atomic<int*> ptrs[kMaxDevices];
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) {
     *st = fail(SPADE_ERR_CUDA, "no current CUDA device");
     return nullptr;
   }
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  int* p = ptrs[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* a = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
     if (e != cudaSuccess) {
       *st = cuda_fail(e, "fixed scratch address");
       return nullptr;
     }
-    ptrs[dev] = static_cast<int*>(p);
+    p = static_cast<int*>(a);
+    ptrs[dev].store(p, std::memory_order_release);
   }
-  return ptrs[dev];
+  return p;
 }
 
 }  // namespace
 
 int num_sms() {
-  static int sms[kMaxDevices] = {0};
+  static std::atomic<int> sms[kMaxDevices];
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return 1;
-  if (!sms[dev]) {
-    int v = 0;
+  int v = sms[dev].load(std::memory_order_relaxed);
+  if (!v) {
     cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    sms[dev] = v > 0 ? v : 1;
+    if (v <= 0) v = 1;
+    sms[dev].store(v, std::memory_order_relaxed);
   }
-  return sms[dev];
+  return v;
 }
 
 long long device_wait_timeout_ns() {
-  static long long ns = -1;
-  if (ns < 0) {
+  static const long long ns = [] {
     const char* e = getenv("SPADE_WAIT_TIMEOUT_MS");
     long long ms = e ? atoll(e) : 10000;
     if (ms <= 0) ms = 10000;
-    ns = ms * 1000000LL;
-  }
+    return ms * 1000000LL;
+  }();
   return ns;
 }
 
@@ -423,6 +449,7 @@ spade_status spade_block_sparse_attn(const void* q, const void* k, const void* v
   a.work = static_cast<int*>(workspace);
   a.n_items = heads * (nb + text_blocks(text_tokens));
   a.ticket = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + need - 256);
+  if ((st = check_attention(a)) != SPADE_OK) return st;
   return run_attention(a, as_cuda(stream));
 }
 
@@ -443,8 +470,6 @@ spade_status spade_block_sparse_attn_noalloc(const void* q, const void* k, const
   if (n_items > SPADE_NOALLOC_MAX_ITEMS)
     return fail(SPADE_ERR_UNSUPPORTED, "heads * (blocks + text blocks) = %lld exceeds the fixed scratch of %d work items",
                 n_items, SPADE_NOALLOC_MAX_ITEMS);
-  int* scratch = noalloc_scratch(&st);
-  if (!scratch) return st;
   AttnArgs a;
   memset(&a, 0, sizeof(a));
   a.q = q; a.k = k; a.v = v; a.out = out;
@@ -459,9 +484,12 @@ spade_status spade_block_sparse_attn_noalloc(const void* q, const void* k, const
     a.head[h].idx_off = (long long)h * nb * nb;
   }
   a.cnt = cnt; a.idx = idx;
+  a.n_items = (int)n_items;
+  if ((st = check_attention(a)) != SPADE_OK) return st;
+  int* scratch = noalloc_scratch(&st);
+  if (!scratch) return st;
   a.work = scratch;                                   // written in full by the work-list kernel
   a.ticket = scratch + SPADE_NOALLOC_MAX_ITEMS;       // reset to 0 by the work-list kernel
-  a.n_items = (int)n_items;
   return run_attention(a, as_cuda(stream));
 }
 
@@ -567,6 +595,30 @@ spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, 
   cudaStream_t s = as_cuda(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int N = schemes[0].T * schemes[0].H * schemes[0].W;
+  // the attention launch of step 5, set up (and checked) before anything is enqueued
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out;
+  a.n_schemes = n_schemes;
+  for (int sc = 0; sc < n_schemes; ++sc) a.geo[sc] = make_geo(schemes[sc]);
+  a.heads = heads; a.d = d; a.text_tokens = text_tokens; a.N = N; a.dt = dt;
+  for (int h = 0; h < heads; ++h) {
+    const int sc = table[h].scheme;
+    const Geo& g = a.geo[sc];
+    a.head[h].scheme = sc;
+    a.head[h].nb = g.nb;
+    a.head[h].dense = table[h].dense;
+    if (!table[h].dense) {
+      a.head[h].cnt_off = (int)((L.cnt[sc] + (size_t)L.pos[h] * g.nb * sizeof(int)) / sizeof(int));
+      a.head[h].idx_off = (long long)((L.idx[sc] + (size_t)L.pos[h] * g.nb * g.nb * sizeof(int)) / sizeof(int));
+    }
+  }
+  a.cnt = reinterpret_cast<const int*>(ws);
+  a.idx = reinterpret_cast<const int*>(ws);
+  a.work = reinterpret_cast<int*>(ws + L.work);
+  a.ticket = reinterpret_cast<int*>(ws + L.ticket);
+  a.n_items = L.n_items;
+  if ((st = check_attention(a)) != SPADE_OK) return st;
   // steps 1-4 per scheme, for its non-dense heads
   for (int sc = 0; sc < n_schemes; ++sc) {
     const int hs = L.n_sparse[sc];
@@ -608,28 +660,6 @@ spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, 
     if (e != cudaSuccess) return cuda_fail(e, "select");
   }
   // step 5: one grouped launch over every head
-  AttnArgs a;
-  memset(&a, 0, sizeof(a));
-  a.q = q; a.k = k; a.v = v; a.out = out;
-  a.n_schemes = n_schemes;
-  for (int sc = 0; sc < n_schemes; ++sc) a.geo[sc] = make_geo(schemes[sc]);
-  a.heads = heads; a.d = d; a.text_tokens = text_tokens; a.N = N; a.dt = dt;
-  for (int h = 0; h < heads; ++h) {
-    const int sc = table[h].scheme;
-    const Geo& g = a.geo[sc];
-    a.head[h].scheme = sc;
-    a.head[h].nb = g.nb;
-    a.head[h].dense = table[h].dense;
-    if (!table[h].dense) {
-      a.head[h].cnt_off = (int)((L.cnt[sc] + (size_t)L.pos[h] * g.nb * sizeof(int)) / sizeof(int));
-      a.head[h].idx_off = (long long)((L.idx[sc] + (size_t)L.pos[h] * g.nb * g.nb * sizeof(int)) / sizeof(int));
-    }
-  }
-  a.cnt = reinterpret_cast<const int*>(ws);
-  a.idx = reinterpret_cast<const int*>(ws);
-  a.work = reinterpret_cast<int*>(ws + L.work);
-  a.ticket = reinterpret_cast<int*>(ws + L.ticket);
-  a.n_items = L.n_items;
   return run_attention(a, s);
 }
 
@@ -651,13 +681,6 @@ spade_status spade_selftest_bounded_wait(int64_t timeout_ns, spade_stream_t stre
   if (!sp) return fail(SPADE_ERR_CUDA, "device status word unavailable");
   cudaError_t e = launch_bounded_wait_selftest(sp, timeout_ns, as_cuda(stream));
   return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "bounded-wait self test");
-}
-
-spade_status spade_selftest_exp2_poly(const float* x, float* y, int n, spade_stream_t stream) {
-  if (!x || !y || n < 0) return fail(SPADE_ERR_INVALID, "null pointer or negative n");
-  if (n == 0) return SPADE_OK;
-  cudaError_t e = launch_exp2_poly_selftest(x, y, n, as_cuda(stream));
-  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "exp2 polynomial self test");
 }
 
 }  // extern "C"

@@ -103,7 +103,6 @@ cudaError_t launch_bounded_wait_selftest(int* status, long long timeout_ns, cuda
 size_t sics_workspace_floats(const Geo* cand, int n_cand, int heads);
 cudaError_t launch_sics(const void* q, const void* k, const Geo* cand, int n_cand, int heads, int d, spade_dtype dt,
                         float* ws, float* scores, int* choice, cudaStream_t s);
-cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int n, cudaStream_t s);
 
 int num_sms();                               // SM count of the current device
 long long device_wait_timeout_ns();          // limit for every bounded device wait

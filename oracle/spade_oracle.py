@@ -23,7 +23,8 @@ summary on gist.science/paper/2608.03335).  The pipeline per attention head:
      exact softmax attention restricted to the kept blocks.  (Online softmax is
      how a kernel evaluates it; the oracle evaluates the definition directly.)
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent (each function below restates the
+one it relies on):
   - token n = (t*H + y)*W + x; tensors [N (+text), heads, d]; batch 1;
   - edge blocks are padded; padded keys never receive weight; padded query
     slots produce no output; block means divide by the number of VALID tokens;

@@ -14,10 +14,28 @@ from spade_workloads import CONFIGS
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _declared():
-    text = open(os.path.join(ROOT, "include", "spade.h")).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(spade_[a-z0-9_]+)\s*\(", text)))
+def _declared(*headers):
+    names = set()
+    for h in headers or (os.path.join(ROOT, "include", "spade.h"),):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(spade_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_library_exports_its_selftest_entry_points():
+    """The test-only entry points (declared in an internal header, not in
+    include/spade.h) are exported too, and nothing else is exported under the
+    spade_ prefix."""
+    lib = _lib.load()
+    internal = os.path.join(ROOT, "input_adaptive_block_b200", "csrc", "spade_selftest.h")
+    names = _declared(internal)
+    assert names == ["spade_selftest_bounded_wait"]
+    for n in names:
+        assert hasattr(lib, n) and n in _lib.SIGNATURES, n
+    public = _declared()
+    assert not set(names) & set(public)
+    assert set(_lib.SIGNATURES) == set(public) | set(names)
 
 
 def test_library_exports_every_declared_symbol():
@@ -178,3 +196,58 @@ def test_fused_form_entry_points_host_validation():
     assert lib.spade_select_scores(fake, taus, fake, fake, 2, 0, None) == _lib.SPADE_ERR_INVALID
     assert lib.spade_select_scores(fake, bad_tau, fake, fake, 2, 10, None) == _lib.SPADE_ERR_INVALID
     assert lib.spade_select_scores(fake, taus, fake, fake, 2000, 10, None) == _lib.SPADE_ERR_UNSUPPORTED
+
+
+def test_noalloc_host_validation():
+    """spade_block_sparse_attn_noalloc refuses, on the host and before it
+    touches the device or its fixed scratch: calls with more work items than
+    the fixed scratch holds, and the same bad arguments the workspace entry
+    point refuses."""
+    lib = _lib.load()
+    fake = ctypes.c_void_p(1 << 20)                 # never dereferenced: validation fails first
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    g = SpadeGeom(21, 45, 80, 2, 8, 8)
+    call = lambda q=fake, cnt=None, idx=None, geom=g, heads=40, d=128, text=0, dt=1: \
+        lib.spade_block_sparse_attn_noalloc(q, fake, fake, fake, cnt, idx, geom, heads, d, text, dt, None)
+    big = SpadeGeom(64, 64, 512, 2, 8, 8)           # 16384 blocks x 8 heads > 65536 work items
+    assert call(geom=big, heads=8) == _lib.SPADE_ERR_UNSUPPORTED
+    assert b"fixed scratch" in lib.spade_last_error_message()
+    assert call(q=None) == _lib.SPADE_ERR_INVALID
+    assert call(q=odd) == _lib.SPADE_ERR_INVALID
+    assert call(cnt=fake) == _lib.SPADE_ERR_INVALID       # cnt without idx
+    assert call(d=96) == _lib.SPADE_ERR_UNSUPPORTED
+    assert call(heads=0) == _lib.SPADE_ERR_UNSUPPORTED
+    assert call(heads=200) == _lib.SPADE_ERR_UNSUPPORTED
+    assert call(text=-1) == _lib.SPADE_ERR_INVALID
+    assert call(dt=7) == _lib.SPADE_ERR_INVALID
+    assert call(geom=SpadeGeom(0, 1, 1, 1, 1, 1)) == _lib.SPADE_ERR_INVALID
+    # blocks above 128 slots take the CUDA-core kernel, which cannot hold them
+    assert call(geom=SpadeGeom(16, 16, 16, 2, 8, 16), heads=1, dt=0) == _lib.SPADE_ERR_UNSUPPORTED
+    assert b"128 slots" in lib.spade_last_error_message()
+
+
+def test_attention_refusals_before_any_launch():
+    """Shapes the attention launch cannot run are refused by every entry point
+    before anything is enqueued (no CUDA call is made, so this runs without a
+    GPU): a head with more than 65536 query blocks (video + text; a work item
+    packs the query block in 16 bits), and blocks above 128 slots on the
+    CUDA-core path."""
+    lib = _lib.load()
+    fake = ctypes.c_void_p(1 << 20)
+    huge = ctypes.c_size_t(1 << 40)
+    flat = SpadeGeom(1, 1, 65535 * 128, 1, 1, 128)   # 65535 blocks of 128 tokens
+    assert lib.spade_block_sparse_attn(fake, fake, fake, fake, None, None, flat, 1, 128, 256, 1, fake, huge,
+                                       None) == _lib.SPADE_ERR_UNSUPPORTED
+    assert b"65536 query blocks" in lib.spade_last_error_message()
+    wide = SpadeGeom(16, 16, 16, 2, 8, 16)          # 256-slot blocks
+    assert lib.spade_block_sparse_attn(fake, fake, fake, fake, None, None, wide, 1, 128, 0, 0, fake, huge,
+                                       None) == _lib.SPADE_ERR_UNSUPPORTED
+    assert b"128 slots" in lib.spade_last_error_message()
+    # the grouped call refuses the same shape before its selection steps
+    gs = (SpadeGeom * 1)(wide)
+    rows = (SpadeHeadScheme * 1)(SpadeHeadScheme(0, 0.9, 0))
+    need = lib.spade_grouped_workspace_bytes(gs, 1, rows, 1, 128, 0)
+    assert need > 0
+    assert lib.spade_grouped_attn(fake, fake, fake, fake, gs, 1, rows, 1, 128, 0, 0, fake, need,
+                                  None) == _lib.SPADE_ERR_UNSUPPORTED
+    assert b"128 slots" in lib.spade_last_error_message()

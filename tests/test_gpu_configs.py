@@ -37,9 +37,15 @@ def _sample_qblocks(wl, h, rng):
     return sorted(int(b) for b in picks)
 
 
-@pytest.mark.parametrize("name", ["tiny", "wan1.3b", "wan14b", "hunyuan", "mixed"])
-def test_full_config(name):
+# Wan-14B is also run at the ends of its tau sweep: 0.8 gives the shortest
+# kept lists, 0.95 the longest, and both move the selection cut the most.
+@pytest.mark.parametrize("name,tau", [("tiny", None), ("wan1.3b", None), ("wan14b", None), ("wan14b", 0.8),
+                                      ("wan14b", 0.95), ("hunyuan", None), ("mixed", None)],
+                         ids=["tiny", "wan1.3b", "wan14b", "wan14b@tau=0.8", "wan14b@tau=0.95", "hunyuan", "mixed"])
+def test_full_config(name, tau):
     wl = get_config(name)
+    if tau is not None:
+        wl = wl.with_tau(tau)
     q, k, v = make_qkv(wl, device="cuda")
     out, _, kept = run_grouped(wl, q, k, v)
     assert torch.isfinite(out.float()).all()
