@@ -8,12 +8,16 @@ block-sparse attention, for every head of the workload.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan14b] [--tau 0.9]
     python bench.py --impl reference ...      # the CPU oracle, timed on host cores
+    python bench.py --sharded ...             # one layer split over the ranks by heads
 
 Prints one JSON line (rank 0).  `value` is the effective throughput in
 TFLOP/s: 4*d FLOPs per evaluated (valid query, valid key) pair, summed over
 the whole layer and all ranks, divided by the max-over-ranks step time.
 Multi-GPU runs (torchrun) give each rank its own layer (independent layers,
-e.g. batch elements): weak scaling, no collective on the data path.
+e.g. batch elements): weak scaling, no collective on the data path.  With
+--sharded the ranks split ONE layer by heads (cost-balanced plan, NCCL
+all-to-all before and after): strong scaling.  The single-GPU run adds a
+short pass over the other configurations (`configs`).
 """
 from __future__ import annotations
 
@@ -402,6 +406,251 @@ def run_reference(args):
     return 0
 
 
+def launches_per_step(table, n_schemes) -> int:
+    """Kernels of one grouped call: per scheme with sparse heads, one Q+K
+    summarize launch per run of consecutive heads, the estimator and the
+    index search; then the work list and the attention."""
+    n = 0
+    for s_id in range(n_schemes):
+        hs = [h for h, (sc, _, dense) in enumerate(table) if sc == s_id and not dense]
+        if hs:
+            n += 1 + sum(1 for a, b in zip(hs, hs[1:]) if b != a + 1) + 2
+    return n + 2 if table else 0
+
+
+def read_kept(api, ws, wl, schemes, table):
+    """Kept lists of every head from a grouped workspace (None for dense heads)."""
+    kept = []
+    for h in range(wl.heads):
+        if wl.head_dense[h]:
+            kept.append(None)
+            continue
+        co, io = api.grouped_head_lists(schemes, table, wl.d, wl.text_tokens, h)
+        nb = wl.schemes[wl.head_scheme[h]].nb
+        cnt = ws[co: co + 4 * nb].view(torch_int32()).cpu().numpy()
+        idx = ws[io: io + 4 * nb * nb].view(torch_int32()).view(nb, nb).cpu().numpy()
+        kept.append([idx[i, : cnt[i]] for i in range(nb)])
+    return kept
+
+
+def torch_int32():
+    import torch
+    return torch.int32
+
+
+def timed(fn, steps, stream):
+    """Mean ms of `steps` back-to-back calls, CUDA events on `stream`."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def attention_only(api, q, k, v, wl, schemes, table, ws, out_ref, steps, stream):
+    """The dominant kernel alone over the layer's own masks: step 5 of the
+    grouped layer (spade_grouped_attn_lists: the work list and the one
+    attention launch), checked bit-equal to the grouped step's output."""
+    import torch
+    out2 = torch.empty_like(q)
+
+    def attn():
+        api.grouped_attn_lists(q, k, v, schemes, table, ws, wl.text_tokens, out=out2)
+    attn()
+    torch.cuda.synchronize()
+    assert torch.equal(out_ref, out2), "attention-only launch differs from the grouped step"
+    return timed(attn, steps, stream)
+
+
+def measure_layer(api, wl, dev, stream, steps, warmup, peaks, selection=True):
+    """One configuration: whole-layer step time, kept-pair FLOPs, the
+    attention launch alone against the bf16 peak, and (single-scheme layers)
+    the selection stages against HBM.  Returns (summary dict, tensors)."""
+    import torch
+    from spade_workloads import make_qkv
+    q, k, v = make_qkv(wl, device=dev)
+    schemes = [s_.as_tuple() for s_ in wl.schemes]
+    table = [(wl.head_scheme[h], wl.head_tau[h], wl.head_dense[h]) for h in range(wl.heads)]
+    ws = torch.zeros(api.grouped_workspace_bytes(schemes, table, wl.d, wl.text_tokens), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty_like(q)
+
+    def step():
+        api.grouped_attn(q, k, v, schemes, table, wl.text_tokens, out=out, workspace=ws)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if api.last_device_status() != 0:
+        raise RuntimeError("device status reports a timed-out wait")
+    kept = read_kept(api, ws, wl, schemes, table)
+    flops = kept_pair_flops(wl, kept)
+    sparse = [h for h in range(wl.heads) if not wl.head_dense[h]]
+    kept_frac = (np.mean([np.mean([len(x) for x in kept[h]]) / wl.schemes[wl.head_scheme[h]].nb
+                          for h in sparse]) if sparse else 1.0)
+    ms = timed(step, steps, stream)
+    attn_ms = attention_only(api, q, k, v, wl, schemes, table, ws, out, steps, stream)
+    ach = flops / (attn_ms * 1e-3) / 1e12
+    res = {"ms_per_layer": ms, "attn_ms": attn_ms, "layer_gflop_kept_pairs": flops / 1e9,
+           "eff_tflops_layer": flops / (ms * 1e-3) / 1e12, "attn_tflops": ach,
+           "attn_frac_bf16": ach / peaks["bf16_tflops"], "block_sparsity": float(1.0 - kept_frac)}
+    if selection and len(wl.schemes) == 1 and not any(wl.head_dense):
+        sel = selection_timing(api, q, k, wl, steps, stream, peaks["hbm_gbs"])
+        res["selection_ms"] = sel["total"]["ms"]
+        res["selection_frac_hbm"] = sel["total"]["frac_hbm"]
+        res["selection_phase_frac_hbm"] = sel["phase"]["frac_hbm"]
+        res["_selection"] = sel
+    return res, (q, k, v, schemes, table, ws, out, kept, flops)
+
+
+SWEEP = (("wan1.3b", 0.9), ("wan14b", 0.8), ("wan14b", 0.95), ("hunyuan", 0.9), ("mixed", None))
+
+
+def config_sweep(api, dev, stream, peaks, steps=5, warmup=3):
+    """The other configurations, one short pass each (same measurements as
+    the headline, fewer steps)."""
+    import torch
+    from spade_workloads import get_config
+    out = {}
+    for name, tau in SWEEP:
+        wl = get_config(name)
+        if tau is not None:
+            wl = wl.with_tau(tau)
+        res, tensors = measure_layer(api, wl, dev, stream, steps, warmup, peaks)
+        res.pop("_selection", None)
+        out[f"{name}@tau={tau}" if tau is not None else f"{name}@per-head tau"] = res
+        del tensors
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_sharded(args):
+    """One layer split over the ranks by heads (sharded.head_sharded_layer):
+    each rank starts from its token slice of Q, K, V (text rows on every
+    rank), exchanges it to the heads of its cost plan, runs the grouped
+    launch and exchanges back.  Strong scaling: the whole job is one layer."""
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from input_adaptive_block_b200 import api
+    from input_adaptive_block_b200.sharded import (grouped_attn_layer, head_costs, head_sharded_layer, plan_heads,
+                                                   token_splits)
+    from spade_workloads import get_config, make_qkv
+    world, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29533")
+    dist.init_process_group("nccl", rank=rank, world_size=world, timeout=timedelta(seconds=120),
+                            device_id=dev)
+    wl = get_config(args.config)
+    tau = args.tau if wl.name != "mixed" else None
+    if tau is not None:
+        wl = wl.with_tau(tau)
+    q, k, v = make_qkv(wl, device=dev)                  # every rank generates the layer, keeps its slice
+    schemes = [s_.as_tuple() for s_ in wl.schemes]
+    table = [(wl.head_scheme[h], wl.head_tau[h], wl.head_dense[h]) for h in range(wl.heads)]
+    splits = token_splits(wl.N, world)
+    s0 = sum(splits[:rank])
+    rows = torch.cat([torch.arange(s0, s0 + splits[rank]), torch.arange(wl.N, wl.n_total)]).to(dev)
+    ql, kl, vl = (t.index_select(0, rows).contiguous() for t in (q, k, v))
+    stream = torch.cuda.current_stream(dev)
+
+    def make_plan(kept_frac):
+        return plan_heads(head_costs(wl.N, wl.text_tokens, wl.d, table, kept_frac), world)
+
+    def run(plan):
+        mine = [table[h] for h in plan[rank]]
+        ws = torch.zeros(max(api.grouped_workspace_bytes(schemes, mine, wl.d, wl.text_tokens), 256) if mine
+                         else 256, dtype=torch.uint8, device=dev)
+        fn = grouped_attn_layer(schemes, table, wl.text_tokens, workspace=ws)
+        return (lambda: head_sharded_layer(ql, kl, vl, fn, plan, splits, wl.text_tokens)), ws
+    # first pass on the tau prior, then re-plan from the kept fractions it measured
+    plan = make_plan(None)
+    f, ws = run(plan)
+    f()
+    torch.cuda.synchronize()
+    frac = torch.zeros(wl.heads, dtype=torch.float64, device=dev)
+    mine_rows = [table[h] for h in plan[rank]]
+    for lh, h in enumerate(plan[rank]):
+        if not wl.head_dense[h]:
+            co, _ = api.grouped_head_lists(schemes, mine_rows, wl.d, wl.text_tokens, lh)
+            nb = wl.schemes[wl.head_scheme[h]].nb
+            frac[h] = ws[co: co + 4 * nb].view(torch.int32).double().sum() / (nb * nb)
+    dist.all_reduce(frac)                                # each head's fraction comes from one rank
+    kept_frac = [None if wl.head_dense[h] else float(frac[h]) for h in range(wl.heads)]
+    plan = make_plan(kept_frac)
+    f, ws = run(plan)
+    for _ in range(args.warmup):
+        f()
+    torch.cuda.synchronize()
+    # FLOPs of the layer: every head counted once (on the rank that ran it)
+    mine_rows = [table[h] for h in plan[rank]]
+    fl = 0
+    for lh, h in enumerate(plan[rank]):
+        sc = wl.schemes[wl.head_scheme[h]]
+        vc = _valid_counts(sc)
+        n = int(vc.sum()) + wl.text_tokens
+        if wl.head_dense[h]:
+            fl += 4 * wl.d * n * n
+            continue
+        co, io = api.grouped_head_lists(schemes, mine_rows, wl.d, wl.text_tokens, lh)
+        nb = sc.nb
+        cnt = ws[co: co + 4 * nb].view(torch.int32).cpu().numpy()
+        idx = ws[io: io + 4 * nb * nb].view(torch.int32).view(nb, nb).cpu().numpy()
+        csum = np.array([vc[idx[i, : cnt[i]]].sum() for i in range(nb)])
+        fl += 4 * wl.d * (int((vc * (csum + wl.text_tokens)).sum()) + wl.text_tokens * n)
+    fl_t = torch.tensor([float(fl)], dtype=torch.float64, device=dev)
+    dist.all_reduce(fl_t)
+    flops = float(fl_t.item())
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms = timed(f, args.steps, stream)
+    dist.barrier()
+    ms = reduce_max(ms, world, dev)
+    costs = head_costs(wl.N, wl.text_tokens, wl.d, table, kept_frac)
+    loads = [sum(costs[h] for h in p_) for p_ in plan]
+    extra = {"ms_per_layer": ms, "layer_gflop_kept_pairs": flops / 1e9, "clocks": clk.summary(),
+             "head_plan": {"heads_per_rank": [len(p_) for p_ in plan],
+                           "cost_imbalance": max(loads) / (sum(loads) / len(loads)) - 1.0,
+                           "rule": "LPT on measured kept fractions (dense heads 4 d (N+text)^2)"},
+             "gpu_launches": args.steps * launches_per_step([table[h] for h in plan[rank]], len(wl.schemes)),
+             "exchange": "torch.distributed all_to_all_single (NCCL) before and after the layer"}
+    if not args.no_e2e:
+        # host token slices in (pinned), the sharded layer, the output slice back
+        hq, hk, hv = (t.cpu().pin_memory() for t in (ql, kl, vl))
+        ho = torch.empty(ql.shape, dtype=ql.dtype).pin_memory()
+        dq, dk, dv = (torch.empty_like(t) for t in (ql, kl, vl))
+
+        def e2e():
+            for d_, h_ in ((dq, hq), (dk, hk), (dv, hv)):
+                d_.copy_(h_, non_blocking=True)
+            o = head_sharded_layer(dq, dk, dv, grouped_attn_layer(schemes, table, wl.text_tokens, workspace=ws),
+                                   plan, splits, wl.text_tokens)
+            ho.copy_(o, non_blocking=True)
+        e2e()
+        torch.cuda.synchronize()
+        dist.barrier()
+        ems = reduce_max(timed(e2e, max(1, min(args.steps, 5)), stream), world, dev)
+        extra["e2e"] = {"value": flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+                        "h2d_bytes_per_step": world * 3 * ql.numel() * ql.element_size(),
+                        "d2h_bytes_per_step": world * ql.numel() * ql.element_size(), "ms_per_step": ems,
+                        "call": "pinned token slices -> head_sharded_layer -> pinned output slice, per rank"}
+    if rank == 0:
+        cfg = workload_config(wl, tau)
+        cfg["parallelism"] = f"head-sharded over {world} ranks (sequence-sharded in and out)"
+        line = assemble_line(value=flops / (ms * 1e-3) / 1e12, unit="TFLOP/s", n_gpus=world, steps=args.steps,
+                             warmup=args.warmup, ms=ms, config=cfg, extra=extra)
+        line["scaling"] = "strong"
+        print(json.dumps(line))
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -410,170 +659,107 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="wan14b")
     ap.add_argument("--tau", type=float, default=0.9)
+    ap.add_argument("--sharded", action="store_true",
+                    help="one layer split over the ranks by heads (strong scaling) instead of one layer per rank")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the short pass over the other configurations")
     ap.add_argument("--e2e-chunk", type=int, default=4, help="heads per pipelined group in the e2e call")
-    ap.add_argument("--e2e-slots", type=int, default=3, help="device group slots in the e2e call")
-    ap.add_argument("--e2e-streams", type=int, default=2, help="compute streams in the e2e call")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.sharded:
+        return run_sharded(args)
 
     import torch
     import torch.distributed as dist
     from input_adaptive_block_b200 import api
-    from spade_workloads import get_config, make_qkv
+    from spade_workloads import get_config
 
     world, rank, local = _dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     wl = get_config(args.config)
     tau = args.tau if wl.name != "mixed" else None
     if tau is not None:
         wl = wl.with_tau(tau)
-    q, k, v = make_qkv(wl, device=dev)
-    schemes = [s.as_tuple() for s in wl.schemes]
-    table = [(wl.head_scheme[h], wl.head_tau[h], wl.head_dense[h]) for h in range(wl.heads)]
-    need = api.grouped_workspace_bytes(schemes, table, wl.d, wl.text_tokens)
-    ws = torch.zeros(need, dtype=torch.uint8, device=dev)
-    out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
+    peaks = _peaks()
+    res, (q, k, v, schemes, table, ws, out, kept, flops) = measure_layer(api, wl, dev, stream, args.steps,
+                                                                         args.warmup, peaks, selection=False)
 
     def step():
         api.grouped_attn(q, k, v, schemes, table, wl.text_tokens, out=out, workspace=ws)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if api.last_device_status() != 0:
-        raise RuntimeError("device status reports a timed-out wait")
-
-    # kept lists of this layer (for the FLOP count and the attention-only timing)
-    kept = []
-    for h in range(wl.heads):
-        if wl.head_dense[h]:
-            kept.append(None)
-            continue
-        co, io = api.grouped_head_lists(schemes, table, wl.d, wl.text_tokens, h)
-        nb = wl.schemes[wl.head_scheme[h]].nb
-        cnt = ws[co: co + 4 * nb].view(torch.int32).cpu().numpy()
-        idx = ws[io: io + 4 * nb * nb].view(torch.int32).view(nb, nb).cpu().numpy()
-        kept.append([idx[i, : cnt[i]] for i in range(nb)])
-    flops = kept_pair_flops(wl, kept)
-    sparse = [h for h in range(wl.heads) if not wl.head_dense[h]]
-    kept_frac = (np.mean([np.mean([len(x) for x in kept[h]]) / wl.schemes[wl.head_scheme[h]].nb
-                          for h in sparse]) if sparse else 1.0)
 
     # ---- timed region: K whole-layer steps ----
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize()
+        ms = timed(step, args.steps, stream)
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1) / args.steps
     ms = reduce_max(ms, world, dev)
     value = world * flops / (ms * 1e-3) / 1e12
     clocks = clk.summary()
 
-    # ---- the dominant kernel alone: attention launches over the same masks ----
-    extra = {}
-    if len(wl.schemes) == 1 and not any(wl.head_dense):
-        co, io = api.grouped_head_lists(schemes, table, wl.d, wl.text_tokens, 0)
-        nb = wl.schemes[0].nb
-        cnt_t = ws[co: co + 4 * nb * wl.heads].view(torch.int32).view(wl.heads, nb)
-        idx_t = ws[io: io + 4 * nb * nb * wl.heads].view(torch.int32).view(wl.heads, nb, nb)
-        aws = torch.empty(max(api.attn_workspace_bytes(schemes[0], wl.heads, wl.d, wl.text_tokens), 256),
-                          dtype=torch.uint8, device=dev)
-        out2 = torch.empty_like(q)
-
-        def attn():
-            api.block_sparse_attn(q, k, v, cnt_t, idx_t, schemes[0], wl.text_tokens, out=out2, workspace=aws)
-        attn()
-        torch.cuda.synchronize()
-        assert torch.equal(out, out2), "attention-only launch differs from the grouped step"
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(args.steps):
-            attn()
-        a1.record(stream)
-        torch.cuda.synchronize()
-        attn_ms = a0.elapsed_time(a1) / args.steps
-    else:
-        attn_ms = None
-
-    peaks = _peaks()
-    if attn_ms is not None:
-        ach = flops / (attn_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / peaks["bf16_tflops"], "traffic": attention_traffic(args.config, tau),
-                "kernel": "attn_tc_kernel<128> (+ work-list build) via spade_block_sparse_attn",
-                "peak_source": f"{peaks['source']} bf16 burst (sustained {peaks['bf16_tflops_sustained']})",
-                "attn_ms": attn_ms}
-    else:
-        ach = flops / (ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach / peaks["bf16_tflops"], "traffic": None,
-                "kernel": "whole grouped step (mixed schemes)", "peak_source": f"{peaks['source']} bf16 burst"}
-    extra["roofline"] = roof
+    # ---- the dominant kernel alone: step 5 over the same masks ----
+    attn_ms = res["attn_ms"]
+    ach = flops / (attn_ms * 1e-3) / 1e12
+    extra = {"roofline": {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                          "frac": ach / peaks["bf16_tflops"], "traffic": attention_traffic(args.config, tau),
+                          "kernel": "attn_tc_kernel<128> (+ work-list build) via spade_grouped_attn_lists",
+                          "peak_source": f"{peaks['source']} bf16 burst (sustained {peaks['bf16_tflops_sustained']})",
+                          "attn_ms": attn_ms}}
     if len(wl.schemes) == 1 and not any(wl.head_dense):
         extra["selection"] = selection_timing(api, q, k, wl, args.steps, stream, peaks["hbm_gbs"])
         if wl.text_tokens == 0 and wl.d == 128:
             extra["scheme_generation"] = sics_timing(api, q, k, wl, args.steps, stream, peaks["hbm_gbs"])
     extra["ms_per_layer"] = ms
-    extra["block_kept_fraction"] = float(kept_frac)
-    extra["block_sparsity"] = float(1.0 - kept_frac)
+    extra["block_kept_fraction"] = 1.0 - res["block_sparsity"]
+    extra["block_sparsity"] = res["block_sparsity"]
     extra["layer_gflop_kept_pairs"] = flops / 1e9
-    n_runs = 0
-    for s_id in range(len(wl.schemes)):
-        hs = [h for h in range(wl.heads) if wl.head_scheme[h] == s_id and not wl.head_dense[h]]
-        if hs:
-            runs = 1 + sum(1 for a, b in zip(hs, hs[1:]) if b != a + 1)
-            n_runs += runs + 2          # one Q+K summarize launch per run of heads, scores, select
-    extra["gpu_launches"] = args.steps * (n_runs + 2)
+    extra["gpu_launches"] = args.steps * launches_per_step(table, len(wl.schemes))
     extra["clocks"] = clocks
 
     # ---- end to end: pinned host inputs in, host output back, every step ----
     if not args.no_e2e:
-        # the public call for host-resident layers: pinned Q, K, V in, O out,
-        # streamed through the GPU by head groups (copies overlap compute)
+        # the public call for host-resident layers (spade_grouped_attn_host):
+        # pinned Q, K, V in, O out, streamed through the GPU by head groups on
+        # the library's own streams; its device workspace is allocated once
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hws = torch.empty(api.grouped_host_workspace_bytes(schemes, table, wl.d, wl.text_tokens, q.dtype,
+                                                           args.e2e_chunk), dtype=torch.uint8, device=dev)
 
         def e2e_step():
             api.grouped_attn_from_host(qh, kh, vh, oh, schemes, table, wl.text_tokens, head_chunk=args.e2e_chunk,
-                                       slots=args.e2e_slots, compute_streams=args.e2e_streams)
+                                       workspace=hws)
         e2e_step()
         torch.cuda.synchronize()
+        assert torch.equal(oh, out.cpu()), "host-to-host call differs from the device-resident step"
         if world > 1:
             dist.barrier()
-        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_e2e = max(1, min(args.steps, 5))
-        b0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        b1.record(stream)
-        torch.cuda.synchronize()
-        ems = reduce_max(b0.elapsed_time(b1) / n_e2e, world, dev)
+        ems = reduce_max(timed(e2e_step, max(1, min(args.steps, 5)), stream), world, dev)
         extra["e2e"] = {"value": world * flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
                         "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                         "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": ems,
-                        "call": f"grouped_attn_from_host (pinned host tensors, head groups of {args.e2e_chunk}, "
-                                f"{args.e2e_slots} device slots, {args.e2e_streams} compute streams)"}
+                        "call": f"spade_grouped_attn_host (pinned host tensors, head groups of {args.e2e_chunk}, "
+                                f"workspace allocated once outside the timed region)"}
+        del qh, kh, vh, oh, hws
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         extra["cpu_baseline"] = cpu_baseline(wl, q, k, v, flops)
+
+    if not args.no_sweep and world == 1:
+        del q, k, v, ws, out
+        torch.cuda.empty_cache()
+        extra["configs"] = config_sweep(api, dev, stream, peaks)
 
     if rank == 0:
         line = assemble_line(value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,

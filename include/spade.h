@@ -249,6 +249,18 @@ spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, 
                                    const int* window_radius,
                                    void* workspace, size_t ws_bytes, spade_stream_t stream);
 
+/* Step 5 alone for a grouped layer: the one attention launch over every
+ * head, under the kept lists that an earlier spade_grouped_attn /
+ * spade_grouped_attn_ex call with the same schemes, table, d and text_tokens
+ * left in `workspace` (for instance to reuse a layer's mask on new Q/K/V, or
+ * to time the attention apart from the selection).  Same arguments as
+ * spade_grouped_attn; the workspace's kept lists are read, not written. */
+spade_status spade_grouped_attn_lists(const void* q, const void* k, const void* v, void* out,
+                                      const spade_geom* schemes, int n_schemes,
+                                      const spade_head_scheme* table, int heads, int d,
+                                      int text_tokens, spade_dtype dt,
+                                      void* workspace, size_t ws_bytes, spade_stream_t stream);
+
 /* Where, inside a grouped workspace, head `head`'s kept lists live (byte
  * offsets of its int32 cnt [nb] and idx [nb, nb] arrays); -1 for dense heads.
  * Lets a caller read back the mask the grouped call used. */
@@ -293,6 +305,39 @@ spade_status spade_sics(const void* q, const void* k, const spade_geom* candidat
  * of another. */
 spade_status spade_copy_head_slice(void* device, void* host, int64_t rows, int heads_total, int h0, int hc,
                                    int d, spade_dtype dt, int to_device, spade_stream_t stream);
+
+/* ---- steps 1-5 from host memory to host memory ------------------------------
+ * One layer whose Q/K/V live in host memory and whose output goes back to
+ * host memory.  Every step is per head (Methodology 3, "Head Grouping"), so
+ * the layer is streamed through the GPU in groups of head_chunk heads: group
+ * g is copied in (strided 2-D copies of its head slice) while an earlier
+ * group runs spade_grouped_attn and a finished group is copied out, on
+ * streams of the library's own.  Three device slots hold the groups in
+ * flight and two compute streams alternate, so a group's kernels start on
+ * the SMs the previous group's attention releases.
+ * q_host, k_host, v_host : [N + text_tokens, heads, d] host arrays, dtype dt;
+ *                          page-locked (cudaHostAlloc / cudaHostRegister)
+ *                          for the copies to overlap the compute (pageable
+ *                          memory works, with synchronous copies).
+ * out_host               : [N + text_tokens, heads, d] host array, written.
+ * schemes, table         : as for spade_grouped_attn (table: all heads).
+ * head_chunk             : heads per group, 1 .. heads.
+ * workspace              : device scratch of
+ *                          spade_grouped_host_workspace_bytes() bytes (the
+ *                          slots and one grouped workspace per compute
+ *                          stream); the call allocates nothing.
+ * The work is ordered after what `stream` holds at the call, and `stream`
+ * waits for all of it: out_host is complete once `stream` is.  The library
+ * creates its streams and events once per device and reuses them; calls on
+ * one device from several host threads are enqueued one at a time. */
+size_t spade_grouped_host_workspace_bytes(const spade_geom* schemes, int n_schemes,
+                                          const spade_head_scheme* table, int heads, int d,
+                                          int text_tokens, spade_dtype dt, int head_chunk);
+spade_status spade_grouped_attn_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                                     const spade_geom* schemes, int n_schemes,
+                                     const spade_head_scheme* table, int heads, int d,
+                                     int text_tokens, spade_dtype dt, int head_chunk,
+                                     void* workspace, size_t ws_bytes, spade_stream_t stream);
 
 /* ---- status ---------------------------------------------------------------
  * spade_last_device_status synchronises `stream`, returns the latched device

@@ -45,6 +45,9 @@ SIGNATURES = {
     "spade_grouped_attn": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SpadeGeom), c_int,
                                    POINTER(SpadeHeadScheme), c_int, c_int, c_int, c_int, c_void_p,
                                    c_size_t, c_void_p]),
+    "spade_grouped_attn_lists": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SpadeGeom), c_int,
+                                         POINTER(SpadeHeadScheme), c_int, c_int, c_int, c_int, c_void_p,
+                                         c_size_t, c_void_p]),
     "spade_grouped_head_lists": (c_int, [POINTER(SpadeGeom), c_int, POINTER(SpadeHeadScheme), c_int,
                                          c_int, c_int, c_int, POINTER(c_int64), POINTER(c_int64)]),
     "spade_summarize_mode": (c_int, [c_void_p, c_void_p, SpadeGeom, c_int, c_int, c_int, c_int, c_void_p]),
@@ -58,6 +61,11 @@ SIGNATURES = {
     "spade_sics_workspace_bytes": (c_size_t, [POINTER(SpadeGeom), c_int, c_int]),
     "spade_sics": (c_int, [c_void_p, c_void_p, POINTER(SpadeGeom), c_int, c_int, c_int, c_int, c_void_p, c_void_p,
                            c_void_p, c_size_t, c_void_p]),
+    "spade_grouped_host_workspace_bytes": (c_size_t, [POINTER(SpadeGeom), c_int, POINTER(SpadeHeadScheme), c_int,
+                                                      c_int, c_int, c_int, c_int]),
+    "spade_grouped_attn_host": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(SpadeGeom), c_int,
+                                        POINTER(SpadeHeadScheme), c_int, c_int, c_int, c_int, c_int, c_void_p,
+                                        c_size_t, c_void_p]),
     "spade_last_device_status": (c_int, [c_void_p]),
     "spade_status_string": (ctypes.c_char_p, [c_int]),
     "spade_last_error_message": (ctypes.c_char_p, []),

@@ -19,7 +19,7 @@ __all__ = [
     "attn_workspace_bytes",
     "block_sparse_attn", "block_sparse_attn_noalloc", "grouped_workspace_bytes", "grouped_attn", "grouped_head_lists",
     "last_device_status", "selftest_bounded_wait", "num_blocks", "sics_workspace_bytes", "sics", "select_window",
-    "grouped_attn_from_host",
+    "grouped_attn_from_host", "grouped_host_workspace_bytes", "grouped_attn_lists",
 ]
 
 
@@ -244,80 +244,50 @@ def grouped_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, schemes, tab
     return out
 
 
+def grouped_attn_lists(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, schemes, table, workspace: torch.Tensor,
+                       text_tokens: int = 0, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Step 5 of a grouped layer under the kept lists an earlier grouped_attn
+    call left in `workspace` (same schemes, table, d, text_tokens)."""
+    heads, d = q.shape[1], q.shape[2]
+    gs, rows = _tables(schemes, table)
+    if out is None:
+        out = torch.empty_like(q)
+    check(_lib.load().spade_grouped_attn_lists(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(out, "out"), gs, len(schemes), rows, heads, d, text_tokens,
+        dtype_code(q.dtype), _dev(workspace, "workspace"), workspace.numel(), _stream(stream)),
+        "spade_grouped_attn_lists")
+    return out
+
+
+def grouped_host_workspace_bytes(schemes, table, d: int, text_tokens: int = 0, dtype=torch.bfloat16,
+                                 head_chunk: int = 4) -> int:
+    gs, rows = _tables(schemes, table)
+    return int(_lib.load().spade_grouped_host_workspace_bytes(gs, len(schemes), rows, len(table), d, text_tokens,
+                                                              dtype_code(dtype), head_chunk))
+
+
 def grouped_attn_from_host(qh: torch.Tensor, kh: torch.Tensor, vh: torch.Tensor, out_h: torch.Tensor, schemes,
-                           table, text_tokens: int = 0, head_chunk: int = 4, device=None,
-                           summary=("mean", "mean"), slots: int = 3, compute_streams: int = 2) -> torch.Tensor:
-    """One layer from host memory to host memory, pipelined by head groups.
-
-    qh, kh, vh, out_h: host tensors [N (+text), heads, d] (pinned for the
-    copies to overlap).  Heads are independent in every step, so the layer
-    is streamed through the GPU in groups of head_chunk heads: an upload
-    stream brings group g in (strided 2-D copies, spade_copy_head_slice)
-    while the compute stream runs the grouped launch on an earlier group and
-    a download stream returns finished groups (uploads and downloads use the
-    two directions of the link at once).  Consecutive groups alternate over
-    `compute_streams` compute streams, so a group's kernels can start on the
-    SMs that the previous group's attention launch has already released.
-    Device buffers: `slots` group slots of Q, K, V and O; group g reuses slot
-    g % slots once group g - slots is back on the host.  Returns out_h after the call's work is
-    enqueued; the caller synchronises (or waits on the current stream, which
-    this call joins at the end)."""
-    if slots < 2:
-        raise ValueError("slots must be >= 2")
-    if compute_streams < 1 or compute_streams > slots:
-        raise ValueError("compute_streams must be in 1..slots")
-    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-    rows, heads, d = qh.shape
-    dt = dtype_code(qh.dtype)
-    lib = _lib.load()
-    caller = torch.cuda.current_stream(dev)
-    computes = [caller] + [torch.cuda.Stream(dev) for _ in range(compute_streams - 1)]
-    for c in computes[1:]:
-        c.wait_stream(caller)
-    up = torch.cuda.Stream(dev)
-    down = torch.cuda.Stream(dev)
-    groups = [(h0, min(head_chunk, heads - h0)) for h0 in range(0, heads, head_chunk)]
-    hcmax = max(hc for _, hc in groups)
-    ns = min(slots, len(groups))
-    # slot x (q, k, v, out), each a flat buffer viewed as [rows, hc, d] for the group it holds
-    bufs = [[torch.empty(rows * hcmax * d, dtype=qh.dtype, device=dev) for _ in range(4)] for _ in range(ns)]
-    need = max(grouped_workspace_bytes(schemes, list(table[h0: h0 + hc]), d, text_tokens) for h0, hc in groups)
-    wss = [torch.empty(max(need, 256), dtype=torch.uint8, device=dev) for _ in computes]   # one per compute stream
-    loaded = [torch.cuda.Event() for _ in groups]
-    done = [torch.cuda.Event() for _ in groups]
-    returned = [torch.cuda.Event() for _ in groups]
-
-    def host_ptr(t):
-        return ctypes.c_void_p(t.data_ptr())
-
-    def load(gi):
-        h0, hc = groups[gi]
-        if gi >= ns:
-            up.wait_event(returned[gi - ns])              # the slot's previous group is back on the host
-        for src, dstb in zip((qh, kh, vh), bufs[gi % ns][:3]):
-            check(lib.spade_copy_head_slice(dstb.data_ptr(), host_ptr(src), rows, heads, h0, hc, d, dt, 1,
-                                            up.cuda_stream), "spade_copy_head_slice")
-        loaded[gi].record(up)
-
-    for gi in range(ns - 1):
-        load(gi)
-    for gi, (h0, hc) in enumerate(groups):
-        if gi + ns - 1 < len(groups):
-            load(gi + ns - 1)
-        compute = computes[gi % len(computes)]
-        compute.wait_event(loaded[gi])
-        q, k, v, o = (b[: rows * hc * d].view(rows, hc, d) for b in bufs[gi % ns])
-        out = grouped_attn(q, k, v, schemes, list(table[h0: h0 + hc]), text_tokens, out=o,
-                           workspace=wss[gi % len(computes)], stream=compute, summary=summary)
-        done[gi].record(compute)
-        down.wait_event(done[gi])
-        check(lib.spade_copy_head_slice(out.data_ptr(), host_ptr(out_h), rows, heads, h0, hc, d, dt, 0,
-                                        down.cuda_stream), "spade_copy_head_slice")
-        returned[gi].record(down)
-    for c in computes[1:]:
-        caller.wait_stream(c)
-    caller.wait_stream(down)
-    caller.wait_stream(up)
+                           table, text_tokens: int = 0, head_chunk: int = 4,
+                           workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One layer from host memory to host memory (spade_grouped_attn_host):
+    qh, kh, vh, out_h are host tensors [N (+text), heads, d], pinned for the
+    copies to overlap the compute; the library streams the layer through the
+    GPU in groups of head_chunk heads.  workspace: a device uint8 tensor of
+    grouped_host_workspace_bytes (allocated here when omitted).  Returns
+    out_h once the work is enqueued; it is complete when the current stream
+    (or `stream`) is."""
+    for t, name in ((qh, "q"), (kh, "k"), (vh, "v"), (out_h, "out")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    heads, d = qh.shape[1], qh.shape[2]
+    gs, rows = _tables(schemes, table)
+    if workspace is None:
+        need = grouped_host_workspace_bytes(schemes, table, d, text_tokens, qh.dtype, head_chunk)
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+    check(_lib.load().spade_grouped_attn_host(
+        qh.data_ptr(), kh.data_ptr(), vh.data_ptr(), out_h.data_ptr(), gs, len(schemes), rows, heads, d,
+        text_tokens, dtype_code(qh.dtype), head_chunk, _dev(workspace, "workspace"), workspace.numel(),
+        _stream(stream)), "spade_grouped_attn_host")
     return out_h
 
 

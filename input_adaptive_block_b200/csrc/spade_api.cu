@@ -1,11 +1,13 @@
 // C ABI of the SPADE executor hot path (declared in include/spade.h):
 // argument validation, workspace layout, and the order of launches for the
 // single steps and for the grouped (mixed-scheme) layer.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -205,6 +207,35 @@ spade_status run_attention(AttnArgs& a, cudaStream_t s) {
   return SPADE_OK;
 }
 
+// The attention launch of a grouped layer: every head of the table, kept
+// lists of the sparse heads read from their places in the grouped workspace.
+void grouped_attn_args(const void* q, const void* k, const void* v, void* out, const spade_geom* schemes,
+                       int n_schemes, const spade_head_scheme* table, int heads, int d, int text_tokens,
+                       spade_dtype dt, const GroupLayout& L, uint8_t* ws, AttnArgs& a) {
+  memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v; a.out = out;
+  a.n_schemes = n_schemes;
+  for (int sc = 0; sc < n_schemes; ++sc) a.geo[sc] = make_geo(schemes[sc]);
+  a.heads = heads; a.d = d; a.text_tokens = text_tokens; a.N = schemes[0].T * schemes[0].H * schemes[0].W;
+  a.dt = dt;
+  for (int h = 0; h < heads; ++h) {
+    const int sc = table[h].scheme;
+    const Geo& g = a.geo[sc];
+    a.head[h].scheme = sc;
+    a.head[h].nb = g.nb;
+    a.head[h].dense = table[h].dense;
+    if (!table[h].dense) {
+      a.head[h].cnt_off = (int)((L.cnt[sc] + (size_t)L.pos[h] * g.nb * sizeof(int)) / sizeof(int));
+      a.head[h].idx_off = (long long)((L.idx[sc] + (size_t)L.pos[h] * g.nb * g.nb * sizeof(int)) / sizeof(int));
+    }
+  }
+  a.cnt = reinterpret_cast<const int*>(ws);
+  a.idx = reinterpret_cast<const int*>(ws);
+  a.work = reinterpret_cast<int*>(ws + L.work);
+  a.ticket = reinterpret_cast<int*>(ws + L.ticket);
+  a.n_items = L.n_items;
+}
+
 // Device address of g_noalloc_scratch on the current device.  The name is only
 // a host-side stand-in in host code, so the address is looked up once per
 // device (with that device current) and cached.
@@ -227,6 +258,79 @@ int* noalloc_scratch(spade_status* st) {
     ptrs[dev].store(p, std::memory_order_release);
   }
   return p;
+}
+
+// ---- host-to-host pipelined layer (spade_grouped_attn_host) ----
+constexpr int kHostSlots = 3;        // device group slots in flight
+constexpr int kHostComputes = 2;     // compute streams the groups alternate over
+
+// Layout of the caller's workspace for the host-to-host call.
+struct HostLayout {
+  int heads, head_chunk, n_groups, hc_max;
+  size_t slot_bytes;       // one of Q, K, V, O for the largest group
+  size_t ws_off;           // first grouped workspace
+  size_t ws_bytes;         // each grouped workspace
+  size_t total;
+};
+
+spade_status plan_host(const spade_geom* schemes, int n_schemes, const spade_head_scheme* table, int heads, int d,
+                       int text_tokens, spade_dtype dt, int head_chunk, HostLayout& H) {
+  GroupLayout L;
+  spade_status st = plan_group(schemes, n_schemes, table, heads, d, text_tokens, L);   // the whole table
+  if (st != SPADE_OK) return st;
+  if ((st = check_d_dt(d, dt)) != SPADE_OK) return st;
+  if (head_chunk < 1 || head_chunk > heads) return fail(SPADE_ERR_INVALID, "head_chunk=%d (1..%d)", head_chunk, heads);
+  H.heads = heads;
+  H.head_chunk = head_chunk;
+  H.n_groups = (heads + head_chunk - 1) / head_chunk;
+  H.hc_max = head_chunk;
+  const size_t rows = (size_t)schemes[0].T * schemes[0].H * schemes[0].W + (size_t)text_tokens;
+  const size_t esz = dt == SPADE_BF16 ? 2 : 4;
+  H.slot_bytes = align256(rows * (size_t)H.hc_max * d * esz);
+  H.ws_bytes = 0;
+  for (int g = 0; g < H.n_groups; ++g) {
+    const int h0 = g * head_chunk, hc = std::min(head_chunk, heads - h0);
+    GroupLayout Lg;
+    if ((st = plan_group(schemes, n_schemes, table + h0, hc, d, text_tokens, Lg)) != SPADE_OK) return st;
+    H.ws_bytes = std::max(H.ws_bytes, Lg.total);
+  }
+  H.ws_bytes = align256(H.ws_bytes);
+  const int ns = std::min(kHostSlots, H.n_groups);
+  H.ws_off = (size_t)ns * 4 * H.slot_bytes;
+  H.total = H.ws_off + (size_t)kHostComputes * H.ws_bytes;
+  return SPADE_OK;
+}
+
+// Streams and events of the host-to-host call, created once per device.
+struct HostPipe {
+  std::mutex mu;                    // one call enqueues at a time
+  bool ready = false;
+  cudaStream_t up = nullptr, down = nullptr, comp[kHostComputes] = {nullptr, nullptr};
+  std::vector<cudaEvent_t> ev;      // 3 per group (loaded, done, returned) + joins
+};
+
+HostPipe& host_pipe(int dev) {
+  static HostPipe pipes[kMaxDevices];
+  return pipes[dev];
+}
+
+// Creates the streams, and enough events for n_events (caller holds P.mu).
+cudaError_t host_pipe_setup(HostPipe& P, size_t n_events) {
+  cudaError_t e = cudaSuccess;
+  if (!P.ready) {
+    e = cudaStreamCreateWithFlags(&P.up, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&P.down, cudaStreamNonBlocking);
+    for (int c = 0; e == cudaSuccess && c < kHostComputes; ++c)
+      e = cudaStreamCreateWithFlags(&P.comp[c], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return e;
+    P.ready = true;
+  }
+  while (P.ev.size() < n_events) {
+    cudaEvent_t ev;
+    if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    P.ev.push_back(ev);
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -594,30 +698,9 @@ spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, 
   if (!workspace || ws_bytes < L.total) return fail(SPADE_ERR_WORKSPACE, "workspace needs %zu bytes", L.total);
   cudaStream_t s = as_cuda(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const int N = schemes[0].T * schemes[0].H * schemes[0].W;
   // the attention launch of step 5, set up (and checked) before anything is enqueued
   AttnArgs a;
-  memset(&a, 0, sizeof(a));
-  a.q = q; a.k = k; a.v = v; a.out = out;
-  a.n_schemes = n_schemes;
-  for (int sc = 0; sc < n_schemes; ++sc) a.geo[sc] = make_geo(schemes[sc]);
-  a.heads = heads; a.d = d; a.text_tokens = text_tokens; a.N = N; a.dt = dt;
-  for (int h = 0; h < heads; ++h) {
-    const int sc = table[h].scheme;
-    const Geo& g = a.geo[sc];
-    a.head[h].scheme = sc;
-    a.head[h].nb = g.nb;
-    a.head[h].dense = table[h].dense;
-    if (!table[h].dense) {
-      a.head[h].cnt_off = (int)((L.cnt[sc] + (size_t)L.pos[h] * g.nb * sizeof(int)) / sizeof(int));
-      a.head[h].idx_off = (long long)((L.idx[sc] + (size_t)L.pos[h] * g.nb * g.nb * sizeof(int)) / sizeof(int));
-    }
-  }
-  a.cnt = reinterpret_cast<const int*>(ws);
-  a.idx = reinterpret_cast<const int*>(ws);
-  a.work = reinterpret_cast<int*>(ws + L.work);
-  a.ticket = reinterpret_cast<int*>(ws + L.ticket);
-  a.n_items = L.n_items;
+  grouped_attn_args(q, k, v, out, schemes, n_schemes, table, heads, d, text_tokens, dt, L, ws, a);
   if ((st = check_attention(a)) != SPADE_OK) return st;
   // steps 1-4 per scheme, for its non-dense heads
   for (int sc = 0; sc < n_schemes; ++sc) {
@@ -661,6 +744,121 @@ spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, 
   }
   // step 5: one grouped launch over every head
   return run_attention(a, s);
+}
+
+spade_status spade_grouped_attn_lists(const void* q, const void* k, const void* v, void* out,
+                                      const spade_geom* schemes, int n_schemes, const spade_head_scheme* table,
+                                      int heads, int d, int text_tokens, spade_dtype dt, void* workspace,
+                                      size_t ws_bytes, spade_stream_t stream) {
+  GroupLayout L;
+  spade_status st = plan_group(schemes, n_schemes, table, heads, d, text_tokens, L);
+  if (st != SPADE_OK) return st;
+  if ((st = check_d_dt(d, dt)) != SPADE_OK) return st;
+  if (!q || !k || !v || !out) return fail(SPADE_ERR_INVALID, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+    return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  if (!workspace || ws_bytes < L.total) return fail(SPADE_ERR_WORKSPACE, "workspace needs %zu bytes", L.total);
+  AttnArgs a;
+  grouped_attn_args(q, k, v, out, schemes, n_schemes, table, heads, d, text_tokens, dt, L,
+                    static_cast<uint8_t*>(workspace), a);
+  if ((st = check_attention(a)) != SPADE_OK) return st;
+  return run_attention(a, as_cuda(stream));
+}
+
+size_t spade_grouped_host_workspace_bytes(const spade_geom* schemes, int n_schemes, const spade_head_scheme* table,
+                                          int heads, int d, int text_tokens, spade_dtype dt, int head_chunk) {
+  HostLayout H;
+  if (plan_host(schemes, n_schemes, table, heads, d, text_tokens, dt, head_chunk, H) != SPADE_OK) return 0;
+  return H.total;
+}
+
+spade_status spade_grouped_attn_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                                     const spade_geom* schemes, int n_schemes, const spade_head_scheme* table,
+                                     int heads, int d, int text_tokens, spade_dtype dt, int head_chunk,
+                                     void* workspace, size_t ws_bytes, spade_stream_t stream) {
+  HostLayout H;
+  spade_status st = plan_host(schemes, n_schemes, table, heads, d, text_tokens, dt, head_chunk, H);
+  if (st != SPADE_OK) return st;
+  if (!q_host || !k_host || !v_host || !out_host) return fail(SPADE_ERR_INVALID, "null host pointer");
+  if (!workspace || ws_bytes < H.total) return fail(SPADE_ERR_WORKSPACE, "workspace needs %zu bytes", H.total);
+  if (!aligned16(workspace)) return fail(SPADE_ERR_INVALID, "pointers must be 16-byte aligned");
+  // every group's grouped call is checked before anything is enqueued
+  const int N = schemes[0].T * schemes[0].H * schemes[0].W;
+  for (int g = 0; g < H.n_groups; ++g) {
+    const int h0 = g * head_chunk, hc = std::min(head_chunk, heads - h0);
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.n_schemes = n_schemes;
+    for (int sc = 0; sc < n_schemes; ++sc) a.geo[sc] = make_geo(schemes[sc]);
+    a.heads = hc; a.d = d; a.text_tokens = text_tokens; a.N = N; a.dt = dt;
+    for (int h = 0; h < hc; ++h) {
+      a.head[h].scheme = table[h0 + h].scheme;
+      a.head[h].nb = a.geo[table[h0 + h].scheme].nb;
+      a.head[h].dense = table[h0 + h].dense;
+    }
+    if ((st = check_attention(a)) != SPADE_OK) return st;
+  }
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return fail(SPADE_ERR_CUDA, "no current CUDA device");
+  HostPipe& P = host_pipe(dev);
+  std::lock_guard<std::mutex> lock(P.mu);
+  const int G = H.n_groups, ns = std::min(kHostSlots, G);
+  cudaError_t e = host_pipe_setup(P, (size_t)3 * G + 1 + 2 + kHostComputes);
+  if (e != cudaSuccess) return cuda_fail(e, "stream/event set-up");
+  cudaEvent_t* loaded = P.ev.data();
+  cudaEvent_t* done = loaded + G;
+  cudaEvent_t* returned = done + G;
+  cudaEvent_t* joins = returned + G;            // [0] entry, [1] up, [2] down, [3..] computes
+  const cudaStream_t caller = as_cuda(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int64_t rows = (int64_t)N + text_tokens;
+  const void* src[3] = {q_host, k_host, v_host};
+  // everything below is ordered after the caller's stream at this point
+  if ((e = cudaEventRecord(joins[0], caller)) != cudaSuccess) return cuda_fail(e, "event record");
+  cudaStreamWaitEvent(P.up, joins[0], 0);
+  cudaStreamWaitEvent(P.down, joins[0], 0);
+  for (int c = 0; c < kHostComputes; ++c) cudaStreamWaitEvent(P.comp[c], joins[0], 0);
+  auto slot_buf = [&](int g, int which) { return ws + ((size_t)(g % ns) * 4 + which) * H.slot_bytes; };
+  auto load = [&](int g) -> spade_status {
+    const int h0 = g * head_chunk, hc = std::min(head_chunk, heads - h0);
+    if (g >= ns) cudaStreamWaitEvent(P.up, returned[g - ns], 0);   // the slot's previous group is back
+    for (int t = 0; t < 3; ++t) {
+      spade_status s2 = spade_copy_head_slice(slot_buf(g, t), const_cast<void*>(src[t]), rows, heads, h0, hc, d, dt,
+                                              1, reinterpret_cast<spade_stream_t>(P.up));
+      if (s2 != SPADE_OK) return s2;
+    }
+    const cudaError_t e2 = cudaEventRecord(loaded[g], P.up);
+    return e2 == cudaSuccess ? SPADE_OK : cuda_fail(e2, "event record");
+  };
+  for (int g = 0; g < ns - 1; ++g)
+    if ((st = load(g)) != SPADE_OK) return st;
+  for (int g = 0; g < G; ++g) {
+    if (g + ns - 1 < G && (st = load(g + ns - 1)) != SPADE_OK) return st;
+    const int h0 = g * head_chunk, hc = std::min(head_chunk, heads - h0);
+    const cudaStream_t comp = P.comp[g % kHostComputes];
+    cudaStreamWaitEvent(comp, loaded[g], 0);
+    st = spade_grouped_attn(slot_buf(g, 0), slot_buf(g, 1), slot_buf(g, 2), slot_buf(g, 3), schemes, n_schemes,
+                            table + h0, hc, d, text_tokens, dt, ws + H.ws_off + (size_t)(g % kHostComputes) * H.ws_bytes,
+                            H.ws_bytes, reinterpret_cast<spade_stream_t>(comp));
+    if (st != SPADE_OK) return st;
+    if ((e = cudaEventRecord(done[g], comp)) != cudaSuccess) return cuda_fail(e, "event record");
+    cudaStreamWaitEvent(P.down, done[g], 0);
+    st = spade_copy_head_slice(slot_buf(g, 3), out_host, rows, heads, h0, hc, d, dt, 0,
+                               reinterpret_cast<spade_stream_t>(P.down));
+    if (st != SPADE_OK) return st;
+    if ((e = cudaEventRecord(returned[g], P.down)) != cudaSuccess) return cuda_fail(e, "event record");
+  }
+  // the caller's stream waits for every stream of the call
+  cudaEventRecord(joins[1], P.up);
+  cudaEventRecord(joins[2], P.down);
+  cudaStreamWaitEvent(caller, joins[1], 0);
+  cudaStreamWaitEvent(caller, joins[2], 0);
+  for (int c = 0; c < kHostComputes; ++c) {
+    cudaEventRecord(joins[3 + c], P.comp[c]);
+    cudaStreamWaitEvent(caller, joins[3 + c], 0);
+  }
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SPADE_OK : cuda_fail(e, "host-to-host layer");
 }
 
 spade_status spade_last_device_status(spade_stream_t stream) {

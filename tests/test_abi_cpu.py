@@ -251,3 +251,29 @@ def test_attention_refusals_before_any_launch():
     assert lib.spade_grouped_attn(fake, fake, fake, fake, gs, 1, rows, 1, 128, 0, 0, fake, need,
                                   None) == _lib.SPADE_ERR_UNSUPPORTED
     assert b"128 slots" in lib.spade_last_error_message()
+
+
+def test_host_layer_and_lists_host_validation():
+    """spade_grouped_attn_host and spade_grouped_attn_lists check their
+    arguments and workspace on the host before any CUDA call."""
+    lib = _lib.load()
+    wl, gs, rows = _mixed_tables()
+    fake = ctypes.c_void_p(1 << 20)                 # never dereferenced: validation fails first
+    need = lib.spade_grouped_host_workspace_bytes(gs, 3, rows, wl.heads, wl.d, 0, 1, 4)
+    assert need >= 3 * 4 * wl.N * 4 * wl.d * 2       # three slots of Q, K, V, O for four heads
+    assert lib.spade_grouped_host_workspace_bytes(gs, 3, rows, wl.heads, wl.d, 0, 1, 0) == 0
+    assert lib.spade_grouped_host_workspace_bytes(gs, 3, rows, wl.heads, wl.d, 0, 1, wl.heads + 1) == 0
+    assert lib.spade_grouped_host_workspace_bytes(gs, 3, rows, wl.heads, wl.d, 0, 1, 8) > need
+    call = lambda q=fake, ws=fake, wsb=need, chunk=4: lib.spade_grouped_attn_host(
+        q, fake, fake, fake, gs, 3, rows, wl.heads, wl.d, 0, 1, chunk, ws, wsb, None)
+    assert call(q=None) == _lib.SPADE_ERR_INVALID
+    assert call(wsb=16) == _lib.SPADE_ERR_WORKSPACE
+    assert call(ws=None) == _lib.SPADE_ERR_WORKSPACE
+    assert call(chunk=0) == _lib.SPADE_ERR_INVALID
+    assert call(ws=ctypes.c_void_p((1 << 20) + 8)) == _lib.SPADE_ERR_INVALID
+    gneed = lib.spade_grouped_workspace_bytes(gs, 3, rows, wl.heads, wl.d, 0)
+    lists = lambda q=fake, ws=fake, wsb=gneed: lib.spade_grouped_attn_lists(
+        q, fake, fake, fake, gs, 3, rows, wl.heads, wl.d, 0, 1, ws, wsb, None)
+    assert lists(q=None) == _lib.SPADE_ERR_INVALID
+    assert lists(wsb=gneed - 1) == _lib.SPADE_ERR_WORKSPACE
+    assert lists(q=ctypes.c_void_p((1 << 20) + 4)) == _lib.SPADE_ERR_INVALID

@@ -69,3 +69,15 @@ def test_kept_pair_flops_matches_oracle_pair_count(text):
     pairs = O.kept_token_pairs([sc.as_tuple(), wl.schemes[1].as_tuple()], [kept0, None], text)
     assert flops == 4 * wl.d * pairs
     assert (bench._valid_counts(sc) == O.valid_counts(sc.as_tuple())).all()
+
+
+def test_launches_per_step():
+    """Kernels of one grouped call, counted from the head table."""
+    wl = get_config("mixed")
+    table = [(wl.head_scheme[h], wl.head_tau[h], wl.head_dense[h]) for h in range(wl.heads)]
+    # dense heads: no selection; two sparse schemes, one run of heads each: (1 + 2) x 2, + work list + attention
+    assert bench.launches_per_step(table, 3) == 8
+    assert bench.launches_per_step([(0, 0.9, False)] * 40, 1) == 5
+    # a run of heads broken in two by a dense head: two summarize launches
+    assert bench.launches_per_step([(0, 0.9, False), (0, 0.9, True), (0, 0.9, False)], 1) == 6
+    assert bench.launches_per_step([(0, 0.9, True)] * 3, 1) == 2
