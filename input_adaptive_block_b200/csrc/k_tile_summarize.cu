@@ -151,6 +151,14 @@ __global__ void __launch_bounds__(256, 5) summarize_kernel(const uint8_t* __rest
 // group of 64 (a warp covers 1 KB of the token row) and reads both with one
 // 32-byte load per token: half the load instructions and pointer steps per
 // byte.  Used when every row start is 32-byte aligned.
+//
+// Small layers have too few (block, chunk group) units to keep enough loads
+// in flight with one warp per unit, so each unit's tokens can be split into
+// S consecutive slices taken by S warps of one CTA (S = 1, 2, 4 or 8; the
+// CTA's 8 warps hold 8 / S units per round).  The slices' partial results
+// are combined through shared memory in slice order, so the result is
+// deterministic and depends only on S, which the launcher derives from the
+// geometry and the head range alone.
 __device__ __forceinline__ void ld32(uint4& a, uint4& b, const uint8_t* p) {
   asm volatile("ld.global.nc.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
@@ -162,35 +170,44 @@ __global__ void __launch_bounds__(256, 4) summarize_wide_kernel(const uint8_t* _
                                                               const uint8_t* __restrict__ in1,
                                                               float* __restrict__ out0, float* __restrict__ out1,
                                                               Geo g, long long row_bytes, int head_off_bytes,
-                                                              int chunks, int d) {
+                                                              int chunks, int d, int S) {
   constexpr int EPC = BF16 ? 8 : 4;  // elements per 16-byte chunk
-  const int lane = threadIdx.x & 31;
-  const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  __shared__ float part[8][2 * EPC][32];   // per warp: its slice's partial result, element-major
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per_cta = 8 / S;                 // units per CTA round
+  const int slot = warp / S, sl = warp - slot * S;
   const int groups = (chunks + 63) / 64;
   const long long n_units = (long long)g.nb * groups;
   const long long all_units = in1 ? 2 * n_units : n_units;
   const long long sy = (long long)g.W * row_bytes;     // next y row
   const long long st = (long long)g.H * sy;            // next frame
-  for (long long uu = gwarp; uu < all_units; uu += nwarps) {
-    const bool second = uu >= n_units;
+  // the loop runs the same number of rounds on every warp of the CTA (S > 1 synchronises the CTA)
+  for (long long ub = (long long)blockIdx.x * per_cta; ub < all_units; ub += (long long)gridDim.x * per_cta) {
+    const long long uu = ub + slot;
+    const bool active = uu < all_units;
+    const bool second = active && uu >= n_units;
     const long long u = second ? uu - n_units : uu;
     const uint8_t* x = second ? in1 : in0;
     float* out = second ? out1 : out0;
-    const int b = (int)(u / groups);
-    const int c = (int)(u - (long long)b * groups) * 64 + 2 * lane;   // first of the lane's two chunks
+    const int b = active ? (int)(u / groups) : 0;
+    const int c = active ? (int)(u - (long long)b * groups) * 64 + 2 * lane : chunks;   // first of the lane's two
     int t0, y0, x0, et, eh, ew;
     block_box(g, b, t0, y0, x0, et, eh, ew);
     const int nvalid = et * eh * ew;
     float acc0[EPC], acc1[EPC];
 #pragma unroll
     for (int e = 0; e < EPC; ++e) acc0[e] = acc1[e] = MODE == 0 ? 0.f : (MODE == 1 ? -INFINITY : INFINITY);
-    if (c < chunks) {
+    // this warp's slice of the block's tokens, in (t, y, x) order
+    const int per = (nvalid + S - 1) / S;
+    const int i0 = min(nvalid, sl * per), i1 = min(nvalid, i0 + per);
+    if (c < chunks && i0 < i1) {
+      const int area = eh * ew;
+      const int tl0 = i0 / area, r0 = i0 - tl0 * area;
+      int yl = r0 / ew, xl = r0 - (r0 / ew) * ew;
       const uint8_t* ptr = x + head_off_bytes + (long long)c * 16 +
-                           (((long long)t0 * g.H + y0) * g.W + x0) * row_bytes;
+                           (((long long)(t0 + tl0) * g.H + (y0 + yl)) * g.W + (x0 + xl)) * row_bytes;
       const long long wrap_y = sy - (long long)ew * row_bytes;
       const long long wrap_t = st - (long long)eh * sy;
-      int xl = 0, yl = 0;
       auto step = [&]() {
         ptr += row_bytes;
         if (++xl == ew) {
@@ -202,8 +219,9 @@ __global__ void __launch_bounds__(256, 4) summarize_wide_kernel(const uint8_t* _
           }
         }
       };
+      const int n = i1 - i0;
       int i = 0;
-      for (; i + 4 <= nvalid; i += 4) {
+      for (; i + 4 <= n; i += 4) {
         uint4 va[4], vb[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -216,13 +234,34 @@ __global__ void __launch_bounds__(256, 4) summarize_wide_kernel(const uint8_t* _
           accumulate<BF16, MODE>(acc1, vb[r]);
         }
       }
-      for (; i < nvalid; ++i) {
+      for (; i < n; ++i) {
         uint4 va, vb;
         ld32(va, vb, ptr);
         accumulate<BF16, MODE>(acc0, va);
         accumulate<BF16, MODE>(acc1, vb);
         step();
       }
+    }
+    if (S > 1) {
+      // combine the S slices of each unit in slice order (the first warp of the unit writes)
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) {
+        part[warp][e][lane] = acc0[e];
+        part[warp][EPC + e][lane] = acc1[e];
+      }
+      __syncthreads();
+      if (sl == 0) {
+        for (int o = 1; o < S; ++o) {
+#pragma unroll
+          for (int e = 0; e < EPC; ++e) {
+            acc0[e] = combine<MODE>(acc0[e], part[warp + o][e][lane]);
+            acc1[e] = combine<MODE>(acc1[e], part[warp + o][EPC + e][lane]);
+          }
+        }
+      }
+      __syncthreads();
+    }
+    if (sl == 0 && c < chunks) {
       const float inv = MODE == 0 ? 1.0f / (float)nvalid : 1.0f;
       const int e0 = c * EPC;             // element index within the head-range row (both chunks in one head)
       const int h = e0 / d, dd = e0 - h * d;
@@ -266,15 +305,26 @@ cudaError_t launch_summarize_m(const void* x0, const void* x1, float* out0, floa
   const int groups = wide ? (chunks + 63) / 64 : (chunks + 31) / 32;
   const long long units = (long long)g.nb * groups * (x1 ? 2 : 1);
   const long long resident = (wide ? 4LL : 5LL) * num_sms() * 8;      // warps
+  if (wide) {
+    // slices per unit: the fewest (up to 8) with which the units of two
+    // tensors fill the resident warps; a function of one tensor's units only,
+    // so one- and two-tensor launches give identical results
+    const long long one = (long long)g.nb * groups;
+    int S = 1;
+    while (S < 8 && one * S * 2 < resident) S *= 2;
+    const long long per_cta = 8 / S;
+    const long long ctas = (units + per_cta - 1) / per_cta;
+    const long long rounds = (ctas + resident / 8 - 1) / (resident / 8);
+    long long blocks = (ctas + rounds - 1) / rounds;
+    if (blocks < 1) blocks = 1;
+    summarize_wide_kernel<true, MODE><<<(int)blocks, 256, 0, s>>>(a, b, out0, out1, g, row_bytes, (int)head_off,
+                                                                   chunks, d, S);
+    return cudaGetLastError();
+  }
   const long long per_warp = (units + resident - 1) / resident;
   const long long warps = (units + per_warp - 1) / per_warp;
   long long blocks = (warps + 7) / 8;
   if (blocks < 1) blocks = 1;
-  if (wide) {
-    summarize_wide_kernel<true, MODE><<<(int)blocks, 256, 0, s>>>(a, b, out0, out1, g, row_bytes, (int)head_off,
-                                                                   chunks, d);
-    return cudaGetLastError();
-  }
   if (dt == SPADE_BF16)
     summarize_kernel<true, MODE><<<(int)blocks, 256, 0, s>>>(a, b, out0, out1, g, row_bytes, h0 * d * esz, chunks, d);
   else
