@@ -253,9 +253,9 @@ class L2Flush:
 def selection_timing(api, q, k, wl, steps, stream, hbm_gbs):
     """Steps 1-4 timed one stage at a time through the public C ABI on the
     bench workload (single scheme), in the form the grouped call runs them:
-    summarize Q and K (one launch, spade_summarize_qk), the estimator's pooled scores
-    (spade_estimate_scores), and the index search with the softmax fused in
-    (spade_select_scores).  L2 is flushed (L2Flush) before every timed
+    summarize Q and K (one launch, spade_summarize_qk), the estimator's pooled
+    scores (spade_estimate_scores), and the index search with the softmax
+    fused in (spade_select_scores).  L2 is flushed (L2Flush) before every timed
     call, so each stage reads its inputs from HBM.  Algorithmic bytes:
     summarize reads the two [N, heads, d] tensors and writes two
     [heads, nb, d] fp32 means; the estimator reads both means and writes [heads, nb, nb] fp32
@@ -661,10 +661,12 @@ def main(argv=None):
     ap.add_argument("--tau", type=float, default=0.9)
     ap.add_argument("--sharded", action="store_true",
                     help="one layer split over the ranks by heads (strong scaling) instead of one layer per rank")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="the first H heads of the configuration only (a smaller case of the same layer shape)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the short pass over the other configurations")
-    ap.add_argument("--e2e-chunk", type=int, default=4, help="heads per pipelined group in the e2e call")
+    ap.add_argument("--e2e-chunk", type=int, default=2, help="heads per pipelined group in the e2e call")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -688,6 +690,8 @@ def main(argv=None):
     tau = args.tau if wl.name != "mixed" else None
     if tau is not None:
         wl = wl.with_tau(tau)
+    if args.heads is not None:
+        wl = wl.with_heads(args.heads)
     stream = torch.cuda.current_stream(dev)
     peaks = _peaks()
     res, (q, k, v, schemes, table, ws, out, kept, flops) = measure_layer(api, wl, dev, stream, args.steps,

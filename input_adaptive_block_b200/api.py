@@ -260,14 +260,14 @@ def grouped_attn_lists(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scheme
 
 
 def grouped_host_workspace_bytes(schemes, table, d: int, text_tokens: int = 0, dtype=torch.bfloat16,
-                                 head_chunk: int = 4) -> int:
+                                 head_chunk: int = 2) -> int:
     gs, rows = _tables(schemes, table)
     return int(_lib.load().spade_grouped_host_workspace_bytes(gs, len(schemes), rows, len(table), d, text_tokens,
                                                               dtype_code(dtype), head_chunk))
 
 
 def grouped_attn_from_host(qh: torch.Tensor, kh: torch.Tensor, vh: torch.Tensor, out_h: torch.Tensor, schemes,
-                           table, text_tokens: int = 0, head_chunk: int = 4,
+                           table, text_tokens: int = 0, head_chunk: int = 2,
                            workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """One layer from host memory to host memory (spade_grouped_attn_host):
     qh, kh, vh, out_h are host tensors [N (+text), heads, d], pinned for the

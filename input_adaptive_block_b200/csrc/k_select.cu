@@ -94,41 +94,19 @@ __device__ __forceinline__ int find_bin(const uint32_t* bins, uint32_t r, int la
   return 32 * L + K;
 }
 
-// NPL: blocks per lane (lane owns j = lane*NPL .. lane*NPL + NPL - 1).
+// The index search of one row whose values (scores or probabilities) are in
+// x[] -- lane owns blocks j = lane*NPL .. lane*NPL + NPL - 1, read as -inf
+// (scores) or 0 (probabilities) past nb -- for row i of head h: writes the
+// kept ids (ascending) to idx_row and their number to *cnt_out.  bins: the
+// warp's 1024 shared-memory bins; cb: the warp's NPL * 32 words of
+// shared-memory stage.  vec: idx_row is 16-byte aligned (nb % 4 == 0).
 // WIN: the static window of block radii (rt, ry, rx) around i replaces the
 // diagonal: its blocks are kept first and their mass counts toward tau.
-// SCORES: `in` holds scores (softmax formed here) instead of probabilities.
-// vec: rows of `in` and `idx` are 16-byte aligned (nb % 4 == 0).
+// SCORES: x holds scores (softmax formed here) instead of probabilities.
 template <int NPL, bool WIN, bool SCORES>
-__global__ void __launch_bounds__(kSelWarps * 32, NPL > 24 ? 6 : 8) select_kernel(const float* __restrict__ in,
-                                                                  const __grid_constant__ SelectTaus taus,
-                                                                  int* __restrict__ cnt, int* __restrict__ idx,
-                                                                  int heads, int nb, int vec) {
-  __shared__ __align__(16) uint32_t sbuf[kSelWarps][NPL * 32];   // compacted keys, then the output stage
-  __shared__ __align__(16) uint32_t sbin[kSelWarps][kBins];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * kSelWarps + warp;
-  if (row >= (long long)heads * nb) return;
-  const int h = (int)(row / nb);
-  const int i = (int)(row - (long long)h * nb);
-  const float* prow = in + row * nb;
+__device__ __forceinline__ void select_row(float (&x)[NPL], const SelectTaus& taus, int h, int i, int nb, int vec,
+                                           uint32_t* bins, uint32_t* cb, int* cnt_out, int* idx_row, int lane) {
   const int j0 = lane * NPL;
-  // blocks past nb read as -inf (scores: exp gives 0) or 0 (probabilities),
-  // so the passes below need no per-block range test
-  const float pad = SCORES ? -INFINITY : 0.f;
-  float x[NPL];
-  if (vec) {
-#pragma unroll
-    for (int q = 0; q < NPL / 4; ++q) {
-      float4 v = make_float4(pad, pad, pad, pad);
-      if (j0 + 4 * q < nb) v = __ldg(reinterpret_cast<const float4*>(prow + j0) + q);
-      x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < NPL; ++e) x[e] = j0 + e < nb ? __ldg(prow + j0 + e) : pad;
-  }
-  uint32_t* bins = sbin[warp];
   zero_bins(bins, lane);                           // while the row is in flight
   float scale = kMassOne, pmul = 1.0f;
   if (SCORES) {
@@ -215,7 +193,6 @@ __global__ void __launch_bounds__(kSelWarps * 32, NPL > 24 ? 6 : 8) select_kerne
     const uint32_t inc = warp_incl(mc, lane);
     const int n1 = (int)__shfl_sync(kFull, inc, 31);
     uint32_t at = inc - mc;
-    uint32_t* cb = sbuf[warp];
 #pragma unroll
     for (int e = 0; e < NPL; ++e)
       if ((key[e] - lo - 1u) < (1u << kOctShift)) cb[at++] = key[e];
@@ -296,13 +273,13 @@ __global__ void __launch_bounds__(kSelWarps * 32, NPL > 24 ? 6 : 8) select_kerne
   const uint32_t oinc = warp_incl(mine, lane);
   const int total = (int)__shfl_sync(kFull, oinc, 31);
   uint32_t at = oinc - mine;
-  uint32_t* ob = sbuf[warp];
+  uint32_t* ob = cb;
   __syncwarp();                                    // the compacted keys have been read
 #pragma unroll
   for (int e = 0; e < NPL; ++e)
     if (keep & (1u << e)) ob[at++] = (uint32_t)(j0 + e);
   __syncwarp();
-  int* out = idx + row * nb;
+  int* out = idx_row;
   if (vec) {
     for (int c = 4 * lane; c < total; c += 128) {
       if (c + 4 <= total) {
@@ -314,7 +291,43 @@ __global__ void __launch_bounds__(kSelWarps * 32, NPL > 24 ? 6 : 8) select_kerne
   } else {
     for (int c = lane; c < total; c += 32) out[c] = (int)ob[c];
   }
-  if (lane == 0) cnt[row] = total;
+  if (lane == 0) *cnt_out = total;
+  __syncwarp();                                    // the stage and bins are free for the warp's next row
+}
+
+// NPL: blocks per lane (lane owns j = lane*NPL .. lane*NPL + NPL - 1).
+// WIN, SCORES: as for select_row.  vec: rows of `in` and `idx` are 16-byte
+// aligned (nb % 4 == 0).
+template <int NPL, bool WIN, bool SCORES>
+__global__ void __launch_bounds__(kSelWarps * 32, NPL > 24 ? 6 : 8) select_kernel(const float* __restrict__ in,
+                                                                  const __grid_constant__ SelectTaus taus,
+                                                                  int* __restrict__ cnt, int* __restrict__ idx,
+                                                                  int heads, int nb, int vec) {
+  __shared__ __align__(16) uint32_t sbuf[kSelWarps][NPL * 32];   // compacted keys, then the output stage
+  __shared__ __align__(16) uint32_t sbin[kSelWarps][kBins];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kSelWarps + warp;
+  if (row >= (long long)heads * nb) return;
+  const int h = (int)(row / nb);
+  const int i = (int)(row - (long long)h * nb);
+  const float* prow = in + row * nb;
+  const int j0 = lane * NPL;
+  // blocks past nb read as -inf (scores: exp gives 0) or 0 (probabilities),
+  // so the passes of select_row need no per-block range test
+  const float pad = SCORES ? -INFINITY : 0.f;
+  float x[NPL];
+  if (vec) {
+#pragma unroll
+    for (int q = 0; q < NPL / 4; ++q) {
+      float4 v = make_float4(pad, pad, pad, pad);
+      if (j0 + 4 * q < nb) v = __ldg(reinterpret_cast<const float4*>(prow + j0) + q);
+      x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < NPL; ++e) x[e] = j0 + e < nb ? __ldg(prow + j0 + e) : pad;
+  }
+  select_row<NPL, WIN, SCORES>(x, taus, h, i, nb, vec, sbin[warp], sbuf[warp], cnt + row, idx + row * nb, lane);
 }
 
 // ------------------------------------------------------------ work list --
@@ -411,13 +424,9 @@ cudaError_t launch_select_t(const float* in, const SelectTaus& t, bool win, bool
   return cudaGetLastError();
 }
 
-}  // namespace
 
-cudaError_t launch_select(const float* in, const float* tau_host, int* cnt, int* idx, int heads, int nb,
-                          cudaStream_t s, const int* radius_host, const Geo* g, bool scores) {
-  // host staging (large), one per calling thread: the launch copies it into
-  // the kernel's parameter buffer, so concurrent callers never share it
-  thread_local SelectTaus t;
+// Fills the per-thread staging of taus (and window radii); returns whether any window is set.
+bool stage_taus(SelectTaus& t, const float* tau_host, int heads, const int* radius_host, const Geo* g) {
   for (int h = 0; h < heads; ++h) t.tau[h] = tau_host[h];
   bool win = false;
   if (radius_host && g) {
@@ -429,6 +438,17 @@ cudaError_t launch_select(const float* in, const float* tau_host, int* cnt, int*
     t.nbh = g->nbh;
     t.nbw = g->nbw;
   }
+  return win;
+}
+
+}  // namespace
+
+cudaError_t launch_select(const float* in, const float* tau_host, int* cnt, int* idx, int heads, int nb,
+                          cudaStream_t s, const int* radius_host, const Geo* g, bool scores) {
+  // host staging (large), one per calling thread: the launch copies it into
+  // the kernel's parameter buffer, so concurrent callers never share it
+  thread_local SelectTaus t;
+  const bool win = stage_taus(t, tau_host, heads, radius_host, g);
   const int vec = (nb % 4 == 0) && (reinterpret_cast<uintptr_t>(in) % 16 == 0) &&
                   (reinterpret_cast<uintptr_t>(idx) % 16 == 0);
   const int npl = (nb + 31) / 32;

@@ -724,12 +724,6 @@ spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, 
       if (e != cudaSuccess) return cuda_fail(e, "summarize");
       i = j;
     }
-    float* prob = reinterpret_cast<float*>(ws + L.prob[sc]);
-    int* st = status_ptr();
-    if (!st) return fail(SPADE_ERR_CUDA, "device status word unavailable");
-    bool scores = false;
-    cudaError_t e = run_estimate(qm, km, prob, hs, g.nb, d, st, false, &scores, s);
-    if (e != cudaSuccess) return cuda_fail(e, "estimate");
     std::vector<float> taus(hs);
     std::vector<int> rad(3 * hs, 0);
     for (int i = 0; i < hs; ++i) {
@@ -737,9 +731,15 @@ spade_status spade_grouped_attn_ex(const void* q, const void* k, const void* v, 
       if (window_radius)
         for (int a = 0; a < 3; ++a) rad[3 * i + a] = window_radius[3 * hl[i] + a];
     }
-    e = launch_select(prob, taus.data(), reinterpret_cast<int*>(ws + L.cnt[sc]),
-                      reinterpret_cast<int*>(ws + L.idx[sc]), hs, g.nb, s, window_radius ? rad.data() : nullptr,
-                      &g, scores);
+    int* cnt_s = reinterpret_cast<int*>(ws + L.cnt[sc]);
+    int* idx_s = reinterpret_cast<int*>(ws + L.idx[sc]);
+    float* prob = reinterpret_cast<float*>(ws + L.prob[sc]);
+    int* st = status_ptr();
+    if (!st) return fail(SPADE_ERR_CUDA, "device status word unavailable");
+    bool scores = false;
+    cudaError_t e = run_estimate(qm, km, prob, hs, g.nb, d, st, false, &scores, s);
+    if (e != cudaSuccess) return cuda_fail(e, "estimate");
+    e = launch_select(prob, taus.data(), cnt_s, idx_s, hs, g.nb, s, window_radius ? rad.data() : nullptr, &g, scores);
     if (e != cudaSuccess) return cuda_fail(e, "select");
   }
   // step 5: one grouped launch over every head

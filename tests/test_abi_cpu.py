@@ -277,3 +277,4 @@ def test_host_layer_and_lists_host_validation():
     assert lists(q=None) == _lib.SPADE_ERR_INVALID
     assert lists(wsb=gneed - 1) == _lib.SPADE_ERR_WORKSPACE
     assert lists(q=ctypes.c_void_p((1 << 20) + 4)) == _lib.SPADE_ERR_INVALID
+
