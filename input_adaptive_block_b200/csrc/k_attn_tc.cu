@@ -599,34 +599,48 @@ __global__ void __launch_bounds__(Cfg<D, NS>::THREADS, 1) attn_tc_kernel(const _
         ptx::mbar_arrive(&md[w]);
         if (l != 0.f && m_seen != m_use) l *= ptx::ex2(m_seen - m_use);
         m_seen = m_use;
-        // p = 2^(s*scale*log2e - m) in four 32-column chunks: FFMA2, exp2
-        // (SFU), row-sum FADD2,
-        // bf16 pack, TMEM store; masked columns are -inf and give 0 (chunks
-        // past a short block's prefix are computed all the same: a branch
-        // between chunks costs more than it saves)
+        // p = 2^(s*scale*log2e - m): FFMA2 over the row, then exp2 (SFU),
+        // row-sum FADD2, bf16 pack and TMEM store in four 32-column chunks;
+        // masked columns are -inf and give 0 (chunks past a short block's
+        // prefix are computed all the same: a branch between chunks costs
+        // more than it saves)
         {
+          // in place over the score row: x = s * scale * log2(e) - m for all
+          // 128 columns (FFMA2), then 2^x chunk by chunk, each chunk's
+          // exponentials issued before the previous chunk's sum, bf16 pack
+          // and TMEM store, so the SFU always has queued work
           const float2 nm2 = make_float2(-m_use, -m_use);
           float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                             make_float2(0.f, 0.f)};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float2 pe[16];
+          for (int c = 0; c < 64; ++c) {
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])),
+                                        sl2x2, nm2);
+            sr[2 * c] = __float_as_uint(x.x);
+            sr[2 * c + 1] = __float_as_uint(x.y);
+          }
+          auto exp_chunk = [&](int q) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-              pe[c] = __ffma2_rn(
-                  make_float2(__uint_as_float(sr[32 * q + 2 * c]), __uint_as_float(sr[32 * q + 2 * c + 1])), sl2x2, nm2);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              pe[c].x = ptx::ex2(pe[c].x);
-              pe[c].y = ptx::ex2(pe[c].y);
-            }
-#pragma unroll
-            for (int c = 0; c < 16; ++c) acc4[c & 3] = __fadd2_rn(acc4[c & 3], pe[c]);
+            for (int c = 0; c < 32; ++c) sr[32 * q + c] = __float_as_uint(ptx::ex2(__uint_as_float(sr[32 * q + c])));
+          };
+          auto finish_chunk = [&](int q) {
             uint32_t pk[16];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) pk[c] = ptx::pack_bf16x2(pe[c].x, pe[c].y);
+            for (int c = 0; c < 16; ++c) {
+              const float2 pv = make_float2(__uint_as_float(sr[32 * q + 2 * c]), __uint_as_float(sr[32 * q + 2 * c + 1]));
+              acc4[c & 3] = __fadd2_rn(acc4[c & 3], pv);
+              pk[c] = ptx::pack_bf16x2(pv.x, pv.y);
+            }
             ptx::tmem_st16_nowait(tS + 16 * q, pk);
-          }
+          };
+          exp_chunk(0);
+          exp_chunk(1);
+          finish_chunk(0);
+          exp_chunk(2);
+          finish_chunk(1);
+          exp_chunk(3);
+          finish_chunk(2);
+          finish_chunk(3);
           const float2 a = __fadd2_rn(__fadd2_rn(acc4[0], acc4[1]), __fadd2_rn(acc4[2], acc4[3]));
           l += a.x + a.y;
         }
