@@ -31,3 +31,19 @@ def test_from_host_equals_device_call(chunk, text):
         torch.cuda.synchronize()
         assert api.last_device_status() == 0
         assert torch.equal(oh, ref.cpu())
+
+
+def test_from_host_fp32_tiny():
+    """The fp32 configuration (CUDA-core attention path) through the host entry."""
+    from spade_workloads import get_config
+    wl = get_config("tiny")
+    q, k, v = make_qkv(wl, device="cuda")
+    schemes = [sc.as_tuple() for sc in wl.schemes]
+    table = [(wl.head_scheme[h], wl.head_tau[h], wl.head_dense[h]) for h in range(wl.heads)]
+    ref = api.grouped_attn(q, k, v, schemes, table, wl.text_tokens)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty(qh.shape, dtype=qh.dtype).pin_memory()
+    api.grouped_attn_from_host(qh, kh, vh, oh, schemes, table, wl.text_tokens, head_chunk=1)
+    torch.cuda.synchronize()
+    assert api.last_device_status() == 0
+    assert torch.equal(oh, ref.cpu())
