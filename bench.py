@@ -329,8 +329,10 @@ def selection_timing(api, q, k, wl, steps, stream, hbm_gbs):
 def sics_timing(api, q, k, wl, steps, stream, hbm_gbs):
     """Scheme generation (spade_sics) on the bench layer with the three
     candidates of the mixed head-wise policy (2x8x8, 1x8x16, 8x4x4): one pass
-    over Q and K per candidate, L2 flushed before each timed call.
-    Algorithmic bytes: n_candidates x (Q + K) read, scores written."""
+    over Q and K for all candidates (their common refinement: 1x4x4 cells in
+    8x8x16 regions), L2 flushed before each timed call.
+    Algorithmic bytes: Q + K read once; the per-block values written and
+    re-read by the reduction (under 0.1 % of that) are left out."""
     import torch
     T, H, W = wl.T, wl.H, wl.W
     cands = [(T, H, W, 2, 8, 8), (T, H, W, 1, 8, 16), (T, H, W, 8, 4, 4)]
@@ -349,7 +351,7 @@ def sics_timing(api, q, k, wl, steps, stream, hbm_gbs):
         torch.cuda.synchronize()
         ts.append(e0.elapsed_time(e1))
     ms = float(np.median(ts))
-    nbytes = len(cands) * 2 * wl.N * wl.heads * wl.d * q.element_size()
+    nbytes = 2 * wl.N * wl.heads * wl.d * q.element_size()
     gbs = nbytes / (ms * 1e-3) / 1e9
     picks = np.bincount(choice.cpu().numpy(), minlength=len(cands)).tolist()
     return {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / hbm_gbs, "candidates": ["2x8x8", "1x8x16", "8x4x4"],

@@ -50,6 +50,16 @@ def test_sics_odd_head_count():
     _check(q, k, [(T, H, W, 2, 4, 4), (T, H, W, 4, 8, 2)])
 
 
+def test_sics_per_candidate_path():
+    """Candidates whose common refinement has more cells than the one-pass
+    kernel keeps on chip (8x4x8 cells of 1x2x2 tokens per 8x8x16 region) run
+    one launch per candidate; same check against the oracle."""
+    T, H, W = 9, 10, 18
+    wl = _wl(T, H, W, 3, 128, "bf16", cid=25)
+    q, k, _ = make_qkv(wl, device="cuda")
+    _check(q, k, [(T, H, W, 1, 2, 16), (T, H, W, 8, 8, 2)])
+
+
 def test_sics_picks_the_constructed_scheme():
     rng = np.random.default_rng(4)
     T, H, W, heads, d = 4, 8, 8, 2, 64
