@@ -18,12 +18,15 @@
 //    computing padded columns, and the softmax masks the columns past it.  No
 //    tiled copy of Q/K/V is ever written.
 //  * tcgen05.mma (kind::f16, bf16 in, fp32 accumulate), issued by one thread.
-//    TMEM (512 columns): S0 | S1 | S2 (fp32 scores; key block g of the CTA
-//    uses buffer g % 3) | O (fp32).  The softmax reads S(g) into registers and
-//    writes P(g) (bf16) over the first half of the same buffer, where P V(g)
-//    reads it; S(g+3) is issued into the buffer once P V(g) has completed.
-//    With three buffers a group never waits for its previous P V before
-//    writing the next P, and two score tiles are normally computed ahead.
+//    TMEM (512 columns): five overlapping score slots of 128 fp32 columns,
+//    64 columns apart (slot k = columns [64 k, 64 k + 128); key block g of the
+//    CTA uses slot g % 5), then O (fp32, columns 384-511).  The softmax reads
+//    S(g) into registers and writes P(g) (bf16) over the first half of its
+//    slot, where P V(g) reads it.  A slot's upper half is the next slot's P
+//    region, so S(g) is issued once S(g-1) is in registers and P V(g-4) has
+//    completed: four blocks of P V -> S slack instead of the three that three
+//    disjoint 128-column buffers would give, and a group never waits for its
+//    previous P V before writing the next P.
 //  * Warp specialisation: warp 0 hands out work and issues TMA loads (one K/V
 //    ring), warp 1 issues the Q K^T MMAs and warp 2 the P V MMAs (so neither
 //    stream's waits hold back the other's issue), warps 4-7 and 8-11 are two
@@ -75,11 +78,13 @@ struct Cfg {
   static constexpr int OFF_LX = OFF_MREF + 4 * 128;               // [2 groups][128 rows] row sums
   static constexpr int OFF_BAR = OFF_LX + 4 * 2 * 128;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;               // barriers + alignment slack
-  // three score buffers: S(g) at 128 (g % 3), g counting the CTA's key
-  // blocks over all its items; P(g) (bf16 pairs) is written over the first 64
-  // columns of its own S buffer
+  // five score slots 64 columns apart: S(g) at 64 (g % 5), g counting the
+  // CTA's key blocks over all its items; P(g) (bf16 pairs) is written over
+  // the first 64 columns of its slot, which the slot before it overlaps
   static constexpr uint32_t COL_S = 0;
+  static constexpr int NSL = 5;                  // score slots, 64 columns apart
   static constexpr uint32_t COL_O = 384;
+  static_assert(COL_S + 64 * (NSL - 1) + 128 <= COL_O && COL_O + D <= 512, "TMEM layout");
   static constexpr uint32_t TMEM_COLS = 512;
   // warpgroup 0: producer, two MMA issuers, one idle warp; warpgroups 1-2:
   // softmax.  Registers per thread after the split (setmaxnreg): the split
@@ -299,16 +304,18 @@ __global__ void __launch_bounds__(Cfg<D, NS>::THREADS, 1) attn_tc_kernel(const _
   uint64_t* kv_empty = bars + NS;
   uint64_t* q_full = bars + 2 * NS;
   uint64_t* q_empty = q_full + 1;
-  uint64_t* s_full = q_full + 2;      // [3] S(g) in TMEM buffer g % 3 (MMA commit)
-  uint64_t* p_full = q_full + 5;      // [3] P(g) written over S(g) (128 threads)
-  uint64_t* buf_free = q_full + 8;    // [3] P V(g) complete: buffer g % 3 may take S(g+3) (MMA commit)
-  uint64_t* md = q_full + 11;         // [2] reference max of block j final (128 threads of its group)
-  uint64_t* o_full = q_full + 13;     // last P V of the item complete
-  uint64_t* o_free = q_full + 14;     // epilogue has read O (256 threads)
-  uint64_t* lx_bar = q_full + 15;     // both groups' final row sums published (256 threads)
-  uint64_t* stage_bar = q_full + 16;  // extent codes of the item staged (256 threads)
-  uint64_t* mma_fin = q_full + 17;    // [2] per MMA warp: all its MMAs complete
-  uint64_t* item_full = q_full + 19;
+  constexpr int NSL = C::NSL;
+  uint64_t* s_full = q_full + 2;              // [NSL] S(g) in slot g % NSL (MMA commit)
+  uint64_t* p_full = s_full + NSL;            // [NSL] P(g) written over the slot's first 64 columns (128 threads)
+  uint64_t* buf_free = p_full + NSL;          // [NSL] P V(g) complete (MMA commit)
+  uint64_t* s_read = buf_free + NSL;          // [NSL] S(g) loaded into registers by its softmax group (128 threads)
+  uint64_t* md = s_read + NSL;                // [2] reference max of block j final (128 threads of its group)
+  uint64_t* o_full = md + 2;                  // last P V of the item complete
+  uint64_t* o_free = o_full + 1;              // epilogue has read O (256 threads)
+  uint64_t* lx_bar = o_free + 1;              // both groups' final row sums published (256 threads)
+  uint64_t* stage_bar = lx_bar + 1;           // extent codes of the item staged (256 threads)
+  uint64_t* mma_fin = stage_bar + 1;          // [2] per MMA warp: all its MMAs complete
+  uint64_t* item_full = mma_fin + 2;
   uint64_t* item_empty = item_full + kItemRing;
   int* item_ring = reinterpret_cast<int*>(item_empty + kItemRing);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_ring + kItemRing);
@@ -333,10 +340,11 @@ __global__ void __launch_bounds__(Cfg<D, NS>::THREADS, 1) attn_tc_kernel(const _
     }
     ptx::mbar_init(q_full, 1);
     ptx::mbar_init(q_empty, 1);
-    for (int b = 0; b < 3; ++b) {
+    for (int b = 0; b < NSL; ++b) {
       ptx::mbar_init(&s_full[b], 1);
       ptx::mbar_init(&p_full[b], 128);
       ptx::mbar_init(&buf_free[b], 1);
+      ptx::mbar_init(&s_read[b], 128);
     }
     ptx::mbar_init(&md[0], 128);
     ptx::mbar_init(&md[1], 128);
@@ -439,9 +447,10 @@ __global__ void __launch_bounds__(Cfg<D, NS>::THREADS, 1) attn_tc_kernel(const _
     // ------------------------------------------------------- MMA issuers --
     // Warp 1 issues the score MMAs S(g) = Q K_g^T, warp 2 the P V(g) MMAs.
     // Each commit tracks only its own warp's MMAs, so each warp blocks only on
-    // its own events: S(g) waits for its K tile and for P V(g-3) to have
-    // completed (buffer g % 3 then no longer holds P(g-3)); P V(g) waits for
-    // P(g) and V_g.  One warp waiting never holds back the other's issue,
+    // its own events: S(g) waits for its K tile, for S(g-1) to be in the
+    // softmax's registers (the lower half of slot g % 5 is the upper half of
+    // the slot before) and for P V(g-4) to have completed (the upper half is
+    // P(g-4)'s region); P V(g) waits for P(g) and V_g.  One warp waiting never holds back the other's issue,
     // which keeps the (shallow) tensor instruction queue fed; a single issuer
     // in a fixed order measured 23 % slower.  Each warp runs in uniform
     // control flow; one elected lane issues each tcgen05.mma / commit.
@@ -452,7 +461,7 @@ __global__ void __launch_bounds__(Cfg<D, NS>::THREADS, 1) attn_tc_kernel(const _
     const bool is_s = warp == 1;
     constexpr uint32_t idesc_pv = make_idesc(128, D, true);
     uint32_t base = 0;         // ring position of the item's first tile
-    uint32_t g = 0;            // key blocks of this warp's stream so far (all items): buffer g % 3
+    uint32_t g = 0;            // key blocks of this warp's stream so far (all items): slot g % 5
     bool ok = true;
     for (int li = 0; ok; ++li) {
       const int slot = li % kItemRing;
@@ -471,16 +480,20 @@ __global__ void __launch_bounds__(Cfg<D, NS>::THREADS, 1) attn_tc_kernel(const _
         ptx::tc_fence_after();
         const uint64_t qdesc = kmajor_desc(ptx::smem_u32(sQ));
         for (int k = 0; ok && k < n; ++k, ++g) {
-          const uint32_t b = g % 3;
+          const uint32_t b = g % NSL;
           const uint32_t pos = base + (uint32_t)(k < 3 ? k : m + 2 * (k - 3) + 1);
           const int st = (int)(pos % NS);
           bool w = wait_bar(&kv_full[st], (pos / NS) & 1, W);
-          // buffer b last held S(g-3) / P(g-3): wait until P V(g-3) has read it
-          if (g >= 3) w = w && wait_bar(&buf_free[b], (g / 3 - 1) & 1, W);
+          // slot b = columns [64 b, 64 b + 128): its upper half is the P region of
+          // slot b + 1, last used by block g - (NSL - 1) -- wait for that P V (which,
+          // in order, also covers P(g - NSL) in the lower half); its lower half is
+          // the upper half of slot b - 1 -- wait until S(g - 1) is in registers
+          if (g >= NSL - 1) w = w && wait_bar(&buf_free[(g + 1) % NSL], ((g - (NSL - 1)) / NSL) & 1, W);
+          if (b != 0) w = w && wait_bar(&s_read[b - 1], ((g - 1) / NSL) & 1, W);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint64_t kdesc = kmajor_desc(ptx::smem_u32(sKV + st * C::TILE));
-          const uint32_t ts = tmem + C::COL_S + 128 * b;
+          const uint32_t ts = tmem + C::COL_S + 64 * b;
           // N = valid key rows rounded up to 16 (the columns past it are masked by the softmax)
           const uint32_t idesc_qk = make_idesc(128, (stage_nv[st] + 15) & ~15, false);
 #pragma unroll
@@ -494,16 +507,16 @@ __global__ void __launch_bounds__(Cfg<D, NS>::THREADS, 1) attn_tc_kernel(const _
         }
       } else {
         for (int j = 0; ok && j < n; ++j, ++g) {
-          const uint32_t b = g % 3;
+          const uint32_t b = g % NSL;
           const uint32_t pos = base + (uint32_t)(m + j + (j < nk3 ? j : nk3));
           const int st = (int)(pos % NS);
-          bool w = wait_bar(&p_full[b], (g / 3) & 1, W);
+          bool w = wait_bar(&p_full[b], (g / NSL) & 1, W);
           w = w && wait_bar(&kv_full[st], (pos / NS) & 1, W);
           if (j == 0) w = w && wait_bar(o_free, (li & 1) ^ 1, W);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint64_t vdesc = mnmajor_desc(ptx::smem_u32(sKV + st * C::TILE));
-          const uint32_t tp = tmem + C::COL_S + 128 * b;   // P(g) over S(g)
+          const uint32_t tp = tmem + C::COL_S + 64 * b;    // P(g) over the first half of S(g)
           const uint32_t acc0 = j > 0 ? 1u : 0u;
           const int nk = (stage_nv[st] + 15) >> 4;       // K steps of 16 keys over the valid prefix
 #pragma unroll 1
@@ -555,14 +568,16 @@ __global__ void __launch_bounds__(Cfg<D, NS>::THREADS, 1) attn_tc_kernel(const _
       float l = 0.f;          // this group's share of the row sum, relative to m_seen
       float m_seen = 0.f;     // reference max at this group's last block
       for (int j = w; j < n; j += 2) {
-        const uint32_t g = g0 + (uint32_t)j;           // the CTA's key-block counter: buffer g % 3
-        const uint32_t b = g % 3;
-        const uint32_t tS = tmem + lane_base + C::COL_S + 128 * b;
-        ok = wait_bar(&s_full[b], (g / 3) & 1, W);
+        const uint32_t g = g0 + (uint32_t)j;           // the CTA's key-block counter: slot g % NSL
+        const uint32_t b = g % NSL;
+        const uint32_t tS = tmem + lane_base + C::COL_S + 64 * b;
+        ok = wait_bar(&s_full[b], (g / NSL) & 1, W);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         ptx::tc_fence_after();
         uint32_t sr[128];
         ptx::tmem_ld128(tS, sr);                       // waits for the loads: P may now overwrite S
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&s_read[b]);                  // S(g+1) may now overwrite the upper half
         const int nv = (int)(sext[j] & 0xffu);         // valid key columns: a prefix
         if (nv < 128) {
 #pragma unroll
@@ -648,7 +663,7 @@ __global__ void __launch_bounds__(Cfg<D, NS>::THREADS, 1) attn_tc_kernel(const _
         if (__any_sync(0xffffffffu, raise)) {
           // O holds blocks < j relative to the old reference: rescale it once
           // P V(j-1) has landed (P V(j) waits for this group's P below)
-          ok = wait_bar(&buf_free[(g - 1) % 3], ((g - 1) / 3) & 1, W);
+          ok = wait_bar(&buf_free[(g - 1) % NSL], ((g - 1) / NSL) & 1, W);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           ptx::tc_fence_after();
 #pragma unroll 1
