@@ -260,18 +260,25 @@ __global__ void __launch_bounds__(256, kFusedMinBlocks) sics_fused_kernel(const 
               }
             }
           }
-          float nq[B], nk[B];       // the raw words stay live, unpacked twice (cheaper than the floats)
+          // squared norms with packed FMAs over element pairs (even and odd
+          // elements summed apart, then added), reduced over the head's lanes;
+          // the raw words stay live and are unpacked again for the sums
+          // (cheaper than keeping the floats across the reductions)
+          float nq[B], nk[B];
 #pragma unroll
           for (int rr = 0; rr < B; ++rr) {
             float xq[EPC], xk[EPC];
             unpack<BF16>(vq[rr], xq);
             unpack<BF16>(vk[rr], xk);
-            nq[rr] = nk[rr] = 0.f;
+            float2 aq = make_float2(0.f, 0.f), ak = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) {
-              nq[rr] = fmaf(xq[e], xq[e], nq[rr]);
-              nk[rr] = fmaf(xk[e], xk[e], nk[rr]);
+            for (int e = 0; e < EPC; e += 2) {
+              const float2 pq = make_float2(xq[e], xq[e + 1]), pk = make_float2(xk[e], xk[e + 1]);
+              aq = __ffma2_rn(pq, pq, aq);
+              ak = __ffma2_rn(pk, pk, ak);
             }
+            nq[rr] = aq.x + aq.y;
+            nk[rr] = ak.x + ak.y;
           }
 #pragma unroll
           for (int o = LPH / 2; o; o >>= 1)
@@ -284,13 +291,18 @@ __global__ void __launch_bounds__(256, kFusedMinBlocks) sics_fused_kernel(const 
           for (int rr = 0; rr < B; ++rr) {
             const float iq = nq[rr] > 0.f ? rsqrtf(nq[rr]) : 0.f;    // zero rows (past the group's share) add nothing
             const float ik = nk[rr] > 0.f ? rsqrtf(nk[rr]) : 0.f;
+            const float2 iq2 = make_float2(iq, iq), ik2 = make_float2(ik, ik);
             float xq[EPC], xk[EPC];
             unpack_again<BF16>(vq[rr], xq);
             unpack_again<BF16>(vk[rr], xk);
 #pragma unroll
-            for (int e = 0; e < EPC; ++e) {
-              uq[e] = fmaf(xq[e], iq, uq[e]);
-              uk[e] = fmaf(xk[e], ik, uk[e]);
+            for (int e = 0; e < EPC; e += 2) {
+              float2 a = __ffma2_rn(make_float2(xq[e], xq[e + 1]), iq2, make_float2(uq[e], uq[e + 1]));
+              uq[e] = a.x;
+              uq[e + 1] = a.y;
+              a = __ffma2_rn(make_float2(xk[e], xk[e + 1]), ik2, make_float2(uk[e], uk[e + 1]));
+              uk[e] = a.x;
+              uk[e + 1] = a.y;
             }
           }
         }

@@ -50,6 +50,16 @@ def test_sics_odd_head_count():
     _check(q, k, [(T, H, W, 2, 4, 4), (T, H, W, 4, 8, 2)])
 
 
+def test_sics_single_token_cells():
+    """Candidates 1x1x2, 1x1x3 and 2x1x1: their common refinement has
+    single-token cells in 2x1x6 regions (a ragged last region along x and
+    t), so every block sums cells of one token."""
+    T, H, W = 3, 5, 20
+    wl = _wl(T, H, W, 3, 128, "bf16", cid=26)
+    q, k, _ = make_qkv(wl, device="cuda")
+    _check(q, k, [(T, H, W, 1, 1, 2), (T, H, W, 1, 1, 3), (T, H, W, 2, 1, 1)])
+
+
 def test_sics_per_candidate_path():
     """Candidates whose common refinement has more cells than the one-pass
     kernel keeps on chip (8x4x8 cells of 1x2x2 tokens per 8x8x16 region) run
