@@ -452,10 +452,30 @@ def timed(fn, steps, stream):
     return e0.elapsed_time(e1) / steps
 
 
-def attention_only(api, q, k, v, wl, schemes, table, ws, out_ref, steps, stream):
+def timed_alternating(fa, fb, steps, stream):
+    """Mean ms of `fa` and of `fb` over `steps` alternating calls (a, b, a,
+    b, ...), each bracketed by its own CUDA events on `stream`, so that both
+    see the same clock under the power cap."""
+    import torch
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        fa()
+        ev[2 * i + 1].record(stream)
+        fb()
+        ev[2 * i + 2].record(stream)
+    torch.cuda.synchronize()
+    ta = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)]
+    tb = [ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(steps)]
+    return float(np.mean(ta)), float(np.mean(tb))
+
+
+def attention_only(api, q, k, v, wl, schemes, table, ws, out_ref, steps, stream, layer_step):
     """The dominant kernel alone over the layer's own masks: step 5 of the
     grouped layer (spade_grouped_attn_lists: the work list and the one
-    attention launch), checked bit-equal to the grouped step's output."""
+    attention launch), checked bit-equal to the grouped step's output, timed
+    in alternation with whole-layer steps.  Returns (layer ms, attention ms)
+    of that alternating pass."""
     import torch
     out2 = torch.empty_like(q)
 
@@ -464,13 +484,15 @@ def attention_only(api, q, k, v, wl, schemes, table, ws, out_ref, steps, stream)
     attn()
     torch.cuda.synchronize()
     assert torch.equal(out_ref, out2), "attention-only launch differs from the grouped step"
-    return timed(attn, steps, stream)
+    return timed_alternating(layer_step, attn, steps, stream)
 
 
 def measure_layer(api, wl, dev, stream, steps, warmup, peaks, selection=True):
-    """One configuration: whole-layer step time, kept-pair FLOPs, the
-    attention launch alone against the bf16 peak, and (single-scheme layers)
-    the selection stages against HBM.  Returns (summary dict, tensors)."""
+    """One configuration: whole-layer step time (`steps` back-to-back
+    steps), kept-pair FLOPs, the attention launch alone against the bf16
+    peak (timed in alternation with layer steps, whose mean is kept as
+    `ms_per_layer_alternating`), and (single-scheme layers) the selection
+    stages against HBM.  Returns (summary dict, tensors)."""
     import torch
     from spade_workloads import make_qkv
     q, k, v = make_qkv(wl, device=dev)
@@ -493,9 +515,10 @@ def measure_layer(api, wl, dev, stream, steps, warmup, peaks, selection=True):
     kept_frac = (np.mean([np.mean([len(x) for x in kept[h]]) / wl.schemes[wl.head_scheme[h]].nb
                           for h in sparse]) if sparse else 1.0)
     ms = timed(step, steps, stream)
-    attn_ms = attention_only(api, q, k, v, wl, schemes, table, ws, out, steps, stream)
+    ms_alt, attn_ms = attention_only(api, q, k, v, wl, schemes, table, ws, out, steps, stream, step)
     ach = flops / (attn_ms * 1e-3) / 1e12
-    res = {"ms_per_layer": ms, "attn_ms": attn_ms, "layer_gflop_kept_pairs": flops / 1e9,
+    res = {"ms_per_layer": ms, "ms_per_layer_alternating": ms_alt, "attn_ms": attn_ms,
+           "layer_gflop_kept_pairs": flops / 1e9,
            "eff_tflops_layer": flops / (ms * 1e-3) / 1e12, "attn_tflops": ach,
            "attn_frac_bf16": ach / peaks["bf16_tflops"], "block_sparsity": float(1.0 - kept_frac)}
     if selection and len(wl.schemes) == 1 and not any(wl.head_dense):
