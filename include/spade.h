@@ -288,6 +288,10 @@ spade_status spade_grouped_head_lists(const spade_geom* schemes, int n_schemes,
  * workspace : device scratch of spade_sics_workspace_bytes() bytes (one
  *             float per head, block and candidate); sums run in a fixed
  *             order, so results are deterministic.
+ * Cost: when the candidates share one T x H x W grid and their common
+ * refinement (cells of the gcd block extents inside regions of the lcm
+ * extents) has at most 64 cells per region, Q and K are read once for all
+ * candidates; otherwise once per candidate.
  * Supported: d in {64, 128}, dt bf16 or f32, heads <= 1024. */
 size_t spade_sics_workspace_bytes(const spade_geom* candidates, int n_candidates, int heads);
 spade_status spade_sics(const void* q, const void* k, const spade_geom* candidates, int n_candidates,
