@@ -750,6 +750,7 @@ def main(argv=None):
         if wl.text_tokens == 0 and wl.d == 128:
             extra["scheme_generation"] = sics_timing(api, q, k, wl, args.steps, stream, peaks["hbm_gbs"])
     extra["ms_per_layer"] = ms
+    extra["ms_per_layer_alternating"] = res["ms_per_layer_alternating"]
     extra["block_kept_fraction"] = 1.0 - res["block_sparsity"]
     extra["block_sparsity"] = res["block_sparsity"]
     extra["layer_gflop_kept_pairs"] = flops / 1e9
