@@ -426,9 +426,10 @@ cudaError_t launch_fused(const void* q, const void* k, float* ws, const SicsFuse
   constexpr int EPC = BF16 ? 8 : 4;
   constexpr int B = kFusedBatch;
   const size_t smem = 2ull * fa.NCT * fa.NCY * fa.NCX * EPC * LPH * sizeof(float);
-  static const cudaError_t attr = cudaFuncSetAttribute(sics_fused_kernel<BF16, LPH, B>,
-                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       (int)(2 * kFusedMaxCells * EPC * LPH * sizeof(float)));
+  // the opt-in is per device, so it is set on every launch (it is cheap)
+  const cudaError_t attr = cudaFuncSetAttribute(sics_fused_kernel<BF16, LPH, B>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)(2 * kFusedMaxCells * EPC * LPH * sizeof(float)));
   if (attr != cudaSuccess) return attr;
   const long long units = (long long)fa.NRT * fa.NRY * fa.NRX * fa.heads;
   long long blocks = units;
