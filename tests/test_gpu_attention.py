@@ -41,6 +41,10 @@ CASES = [
     _wl("text-200", 4, 16, 24, 2, 128, "bf16", (2, 8, 8), text=200),
     _wl("tau1-dense-equivalent", 3, 16, 17, 2, 128, "bf16", (2, 8, 8), tau=1.0),
     _wl("one-block", 1, 4, 4, 2, 128, "bf16", (2, 8, 8)),
+    # tau -> 0: every row keeps its diagonal block only, so the 1152 items
+    # (about eight per persistent CTA) have one key block each and the CTA's
+    # block counter steps through every score slot from item to item
+    _wl("diagonal-only", 8, 48, 64, 6, 128, "bf16", (2, 8, 8), tau=1e-6),
     _mixed_small(),
     get_config("tiny"),
 ]

@@ -60,6 +60,24 @@ def test_sics_single_token_cells():
     _check(q, k, [(T, H, W, 1, 1, 2), (T, H, W, 1, 1, 3), (T, H, W, 2, 1, 1)])
 
 
+def test_sics_four_candidates():
+    """The most candidates a call takes (four), on a ragged grid: their
+    common refinement is 32 cells of 1x2x4 tokens in 4x8x8 regions."""
+    T, H, W = 5, 9, 10
+    wl = _wl(T, H, W, 2, 128, "bf16", cid=27)
+    q, k, _ = make_qkv(wl, device="cuda")
+    _check(q, k, [(T, H, W, 2, 4, 4), (T, H, W, 1, 8, 8), (T, H, W, 4, 2, 4), (T, H, W, 2, 2, 8)])
+
+
+def test_sics_candidates_on_different_grids():
+    """Candidates only need the same number of tokens: here the 192 tokens
+    are read as a 4x6x8 and as an 8x6x4 grid (each candidate walks the token
+    order of its own grid), which takes one pass per candidate."""
+    wl = _wl(4, 6, 8, 2, 64, "bf16", cid=28)
+    q, k, _ = make_qkv(wl, device="cuda")
+    _check(q, k, [(4, 6, 8, 2, 3, 4), (8, 6, 4, 4, 3, 2)])
+
+
 def test_sics_per_candidate_path():
     """Candidates whose common refinement has more cells than the one-pass
     kernel keeps on chip (8x4x8 cells of 1x2x2 tokens per 8x8x16 region) run
